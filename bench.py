@@ -1,0 +1,408 @@
+"""Benchmark: KDA prefill tokens/s (H=32, d=128) and decode-step HBM GB/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0. A "step" is one pass of the hot path over one batch:
+one chunkwise prefill launch over the long-context workload (1,048,576 tokens,
+32 heads, bf16 q/k/v, fp32 gates) -- the headline `value` -- and the decode
+step on its own workload (256 sequences x 32 heads, fp32 state) timed
+separately and reported under "decode".
+
+Multi-GPU: every rank processes its own independent batch (replicas, no
+collective on the data path); value = all ranks' tokens / max-over-ranks time.
+`--impl reference` times the fp64 oracle on the host cores instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import kda_inputs  # noqa: E402
+
+METRIC = "KDA prefill tokens/s (H=32,d=128) & decode-step HBM GB/s vs peak, 1xB200"
+D = 128
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * D + 4 * D + 4 + 2 * D   # q,k,v bf16 + log_alpha f32 + beta + o
+STATE_BYTES = 4 * D * D
+DECODE_BYTES_PER_CHAIN = 2 * STATE_BYTES + 4 * 2 * D + 2 + 2 * D   # state rw + q,k,v,la + beta + o
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while a region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="kda_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _sum_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def _oracle_sample_rate(cfg_idx: int, target_s: float, seed_heads=(0, 1), max_tokens=1 << 20):
+    """Time the fp64 oracle on a bounded sample of a prefill workload.
+
+    Returns (tokens/s scaled to the workload's head count, sample description,
+    threads used, seconds). Throughput scales linearly in heads (heads are
+    independent), so token-heads/s over the sampled heads / n_heads is the
+    oracle's tokens/s for the full head count.
+    """
+    import oracle
+    cfg = kda_inputs.PREFILL_CONFIGS[cfg_idx]
+    H = len(seed_heads)
+    threads = oracle.oracle_threads()
+
+    def run(T):
+        inp = kda_inputs.make_prefill([T], H, cfg.qkv_dtype, torch.float32, cfg.x_mean, cfg.h0,
+                                      cfg.seed, "cpu")
+        t0 = time.perf_counter()
+        oracle.oracle_forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                              h0=inp["h0"], col_block=max(1, D * H // threads))
+        return time.perf_counter() - t0
+
+    T = 2048
+    dt = run(T)
+    T = int(min(max_tokens, max(2048, T * target_s / max(dt, 1e-3))))
+    dt = run(T)
+    rate = T * H / dt / cfg.n_heads
+    desc = (f"{cfg.name}: first {T} tokens of {H} heads (fp64 oracle, {threads} threads), "
+            f"token-heads/s divided by {cfg.n_heads} heads")
+    return rate, desc, threads, dt, T
+
+
+def run_reference(args):
+    """The fp64 oracle on the host cores (rank 0 only)."""
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    cfg = kda_inputs.PREFILL_CONFIGS[3]
+    threads = oracle.oracle_threads()
+    H = 2
+    # calibrate a sample of ~4 s per step
+    _, _, _, _, T = _oracle_sample_rate(3, 4.0)
+    inp = kda_inputs.make_prefill([T], H, cfg.qkv_dtype, torch.float32, cfg.x_mean, cfg.h0,
+                                  cfg.seed, "cpu")
+
+    def step():
+        oracle.oracle_forward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                              col_block=max(1, D * H // threads))
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    rate = args.steps * T * H / dt / cfg.n_heads
+    sample = (f"{cfg.name}: first {T} tokens of {H} heads per step (fp64 oracle), "
+              f"token-heads/s divided by {cfg.n_heads} heads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": 1048576, "H": 32, "d": D, "chunk": 64,
+                   "sampled_T": T, "sampled_heads": H},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def time_prefill(kda, inp, steps, warmup, ws, stream):
+    fwd = lambda: kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], o=inp["o"],
+                                hT=inp["hT"])
+    for _ in range(warmup):
+        fwd()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for a, b in ev:
+        a.record(stream)
+        fwd()
+        b.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch = [a.elapsed_time(b) for a, b in ev]
+    return total_ms, per_launch
+
+
+def time_decode(kda, dec, steps, warmup, stream):
+    n_avail = dec["q"].shape[0]
+    st = dec["state"]
+    o = torch.empty_like(dec["q"][0])
+
+    def step(s):
+        s = s % n_avail
+        kda.decode_step(dec["q"][s], dec["k"][s], dec["v"][s], dec["log_alpha"][s],
+                        dec["beta"][s], st, o=o)
+
+    for s in range(warmup):
+        step(s)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for s in range(steps):
+        step(s)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def time_e2e(kda, inp, steps, stream):
+    """Public API with host buffers: H2D of the step's inputs from pinned memory,
+    the prefill, and D2H of its outputs (o and the final state), every step."""
+    names = ["q", "k", "v", "log_alpha", "beta"]
+    host = {n: torch.empty(inp[n].shape, dtype=inp[n].dtype, pin_memory=True) for n in names}
+    for n in names:
+        host[n].copy_(inp[n])
+    o_host = torch.empty(inp["o"].shape, dtype=inp["o"].dtype, pin_memory=True)
+    h_host = torch.empty(inp["hT"].shape, dtype=inp["hT"].dtype, pin_memory=True)
+    dev = {n: torch.empty_like(inp[n]) for n in names}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = o_host.numel() * o_host.element_size() + h_host.numel() * h_host.element_size()
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        o, hT = kda.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
+                              h0=None, cu_seqlens=inp["cu_seqlens"], o=inp["o"], hT=inp["hT"])
+        o_host.copy_(o, non_blocking=True)
+        h_host.copy_(hT, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    del host, dev, o_host, h_host
+    return ms, h2d, d2h
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    ws, rank, local = _dist()
+    import channel_wise_gated_b200 as kda
+    kda._native.load()   # the in-tree library; raises if missing
+    stream = torch.cuda.current_stream()
+    hbm_peak, bf16_peak, peak_kind = _peaks()
+
+    # ---- prefill workload (each rank its own batch)
+    cfg = kda_inputs.PREFILL_CONFIGS[3]
+    lens = kda_inputs.config_lengths(cfg)
+    inp = kda_inputs.make_prefill(lens, cfg.n_heads, cfg.qkv_dtype, torch.float32, cfg.x_mean,
+                                  cfg.h0, cfg.seed + 100 * rank, "cuda")
+    T, H = sum(lens), cfg.n_heads
+    N = len(lens)
+    inp["o"] = torch.empty_like(inp["q"])
+    inp["hT"] = torch.empty((N, H, D, D), dtype=torch.float32, device="cuda")
+    step_bytes = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + N * H * STATE_BYTES * (
+        2 if inp["h0"] is not None else 1)
+
+    with ClockSampler(local) as clk:
+        total_ms, per_launch = time_prefill(kda, inp, args.steps, args.warmup, ws, stream)
+    clocks = clk.summary()
+    max_ms = _max_over_ranks(total_ms, ws)
+    tokens_all = _sum_over_ranks(float(T * args.steps), ws)
+    value = tokens_all / (max_ms / 1e3)
+    avg_launch_ms = sum(per_launch) / len(per_launch)
+    achieved = step_bytes / (avg_launch_ms / 1e3) / 1e9
+
+    # ---- decode workload
+    dcfg = kda_inputs.DECODE_CONFIG
+    n_pool = 50   # distinct per-step inputs cycled through (all > L2 with the state)
+    dec = kda_inputs.make_decode(dcfg.n_seqs, dcfg.n_heads, n_pool, dcfg.qkv_dtype,
+                                 dcfg.gate_dtype, dcfg.x_mean, dcfg.state_std, dcfg.seed, "cuda")
+    dec_ms = time_decode(kda, dec, args.decode_steps, args.warmup, stream)
+    chains = dcfg.n_seqs * dcfg.n_heads
+    dec_step_us = dec_ms / args.decode_steps * 1e3
+    dec_gbs = chains * DECODE_BYTES_PER_CHAIN / (dec_step_us / 1e6) / 1e9
+    del dec
+    torch.cuda.empty_cache()
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        ms, h2d, d2h = time_e2e(kda, inp, args.e2e_steps, stream)
+        ms = _max_over_ranks(ms, ws)
+        e2e_tokens = _sum_over_ranks(float(T * args.e2e_steps), ws)
+        e2e = {"value": e2e_tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rate, desc, threads, _, _ = _oracle_sample_rate(3, 12.0)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": kda.PREFILL_COMPUTE_DTYPE, "data": "synthetic",
+            "config": {"workload": cfg.name, "T": T, "H": H, "d": D, "chunk": 64,
+                       "qkv": "bf16", "gates": "f32", "state": "f32",
+                       "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB per step)",
+                       "parallelism": f"replicas x{ws}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None,
+                         "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": step_bytes,
+                         "avg_launch_ms": avg_launch_ms},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "decode": {"workload": dcfg.name, "steps": args.decode_steps,
+                       "us_per_step": dec_step_us, "GBps": dec_gbs,
+                       "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak,
+                                    "unit": "GB/s", "frac": dec_gbs / hbm_peak,
+                                    "algorithmic_bytes_per_step": chains * DECODE_BYTES_PER_CHAIN},
+                       "gpu_launches": args.decode_steps,
+                       "l2": "state 512 MiB > L2"},
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,132 @@
+"""Kimi Delta Attention (KDA) on B200: chunkwise prefill and recurrent decode.
+
+Thin Python binding over the C ABI of ``include/kda.h``. PyTorch is used only to
+hold device memory and to name the current CUDA stream; every step of the
+operator runs in the library's CUDA kernels. Functions take torch tensors,
+check their dtypes, shapes and contiguity, and pass raw pointers through.
+
+    o, hT = chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None)
+    o     = decode_step(q, k, v, log_alpha, beta, state)      # state updated in place
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _native
+from ._native import KdaError  # noqa: F401
+
+D = 128
+
+# Arithmetic type of the prefill path's contractions for bf16 inputs.
+PREFILL_COMPUTE_DTYPE = "f32"
+
+_DT = {torch.float32: _native.KDA_F32, torch.bfloat16: _native.KDA_BF16}
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, o=None, hT=None,
+              output_final_state: bool = True, kernel: str = "auto"):
+    """Chunkwise KDA prefill.
+
+    q, k, v: [T, H, 128] bf16 or fp32 (same dtype); log_alpha: [T, H, 128] fp32;
+    beta: [T, H] fp32; h0: [N, H, 128, 128] fp32 or None; cu_seqlens: [N+1] int32
+    on the device or None (one sequence). Returns (o, hT) with o like q and hT
+    [N, H, 128, 128] fp32 (None if output_final_state is False).
+    ``kernel``: "auto" (tensor cores for bf16, CUDA cores for fp32) or "simt"
+    (always the fp32 CUDA-core chunk kernel).
+    """
+    lib = _native.load()
+    if q.dim() != 3 or q.shape[2] != D:
+        raise ValueError("q must be [T, H, 128]")
+    T, H, _ = q.shape
+    dev = q.device
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, (T, H, D), dev)
+    _need(log_alpha, "log_alpha", torch.float32, (T, H, D), dev)
+    _need(beta, "beta", torch.float32, (T, H), dev)
+    if cu_seqlens is None:
+        N = 1
+    else:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be [N+1]")
+        N = cu_seqlens.numel() - 1
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (N, H, D, D), dev)
+    if o is None:
+        o = torch.empty_like(q)
+    else:
+        _need(o, "o", q.dtype, (T, H, D), dev)
+    if output_final_state and hT is None:
+        hT = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
+    elif hT is not None:
+        _need(hT, "hT", torch.float32, (N, H, D, D), dev)
+    fn = lib.kda_chunk_fwd_simt if kernel == "simt" else lib.kda_chunk_fwd
+    if kernel not in ("auto", "simt"):
+        raise ValueError("kernel must be 'auto' or 'simt'")
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
+            N, T, H, _DT[q.dtype], _ptr(o), _ptr(hT), _stream_ptr(dev))
+    _native.check(st, fn.__name__)
+    return o, hT
+
+
+def decode_step(q, k, v, log_alpha, beta, state, o=None):
+    """One recurrent KDA step per (sequence, head), state updated in place.
+
+    q, k, v: [N, H, 128] bf16 or fp32; log_alpha: [N, H, 128], beta: [N, H]
+    (bf16 or fp32, same dtype); state: [N, H, 128, 128] fp32. Returns o like q.
+    """
+    lib = _native.load()
+    if q.dim() != 3 or q.shape[2] != D:
+        raise ValueError("q must be [N, H, 128]")
+    N, H, _ = q.shape
+    dev = q.device
+    if q.dtype not in _DT or log_alpha.dtype not in _DT:
+        raise TypeError("unsupported dtype")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, (N, H, D), dev)
+    _need(log_alpha, "log_alpha", log_alpha.dtype, (N, H, D), dev)
+    _need(beta, "beta", log_alpha.dtype, (N, H), dev)
+    _need(state, "state", torch.float32, (N, H, D, D), dev)
+    if o is None:
+        o = torch.empty_like(q)
+    else:
+        _need(o, "o", q.dtype, (N, H, D), dev)
+    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
+                             _ptr(o), N, H, _DT[q.dtype], _DT[log_alpha.dtype], _stream_ptr(dev))
+    _native.check(st, "kda_decode_step")
+    return o
+
+
+def device_status(device=None) -> int:
+    """Read and clear the library's device-side error word (synchronises)."""
+    lib = _native.load()
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(lib.kda_device_status(_stream_ptr(dev)))

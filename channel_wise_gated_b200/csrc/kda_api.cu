@@ -1,0 +1,158 @@
+// C ABI of the KDA library (declared in include/kda.h): host-side validation and
+// stream-ordered kernel launches. All device code lives in the included headers;
+// this file is the library's single translation unit.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/kda.h"
+#include "kda_chunk_simt.cuh"
+#include "kda_common.cuh"
+#include "kda_decode.cuh"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int validate_chunk_args(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* h0, const int32_t* cu_seqlens,
+                        int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                        const void* o, const float* hT) {
+  if (qkv_dtype != KDA_F32 && qkv_dtype != KDA_BF16) return KDA_ERR_DTYPE;
+  if (n_heads <= 0 || n_seqs <= 0 || t_total < 0) return KDA_ERR_SHAPE;
+  if ((int64_t)n_seqs * n_heads > (int64_t)INT32_MAX / 4) return KDA_ERR_SHAPE;
+  if (cu_seqlens == nullptr && n_seqs != 1) return KDA_ERR_SEQLENS;
+  if (t_total > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, beta, h0, o, hT, cu_seqlens};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_ALIGN;
+  return KDA_OK;
+}
+
+template <typename TQ>
+int launch_chunk_simt(const void* q, const void* k, const void* v, const float* log_alpha,
+                      const float* beta, const float* h0, const int32_t* cu_seqlens,
+                      int32_t n_seqs, int64_t t_total, int32_t n_heads, void* o, float* hT,
+                      cudaStream_t stream) {
+  const size_t smem = sizeof(kda::SimtSmem);
+  if (cudaFuncSetAttribute(kda::chunk_simt_kernel<TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  dim3 grid((unsigned)(n_seqs * n_heads), kda::D / kda::SIMT_DV);
+  kda::chunk_simt_kernel<TQ><<<grid, kda::SIMT_THREADS, smem, stream>>>(
+      static_cast<const TQ*>(q), static_cast<const TQ*>(k), static_cast<const TQ*>(v), log_alpha,
+      beta, h0, cu_seqlens, n_seqs, t_total, n_heads, static_cast<TQ*>(o), hT);
+  return launch_status();
+}
+
+int chunk_simt_dispatch(const void* q, const void* k, const void* v, const float* log_alpha,
+                        const float* beta, const float* h0, const int32_t* cu_seqlens,
+                        int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                        void* o, float* hT, cudaStream_t stream) {
+  if (qkv_dtype == KDA_F32)
+    return launch_chunk_simt<float>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
+                                    n_heads, o, hT, stream);
+  return launch_chunk_simt<__nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs,
+                                          t_total, n_heads, o, hT, stream);
+}
+
+template <typename TQ, typename TG>
+int launch_decode(const void* q, const void* k, const void* v, const void* log_alpha,
+                  const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_heads,
+                  cudaStream_t stream) {
+  const unsigned chains = (unsigned)n_seqs * (unsigned)n_heads;
+  kda::decode_step_kernel<TQ, TG><<<chains, kda::DEC_THREADS, 0, stream>>>(
+      static_cast<const TQ*>(q), static_cast<const TQ*>(k), static_cast<const TQ*>(v),
+      static_cast<const TG*>(log_alpha), static_cast<const TG*>(beta), state, static_cast<TQ*>(o));
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_chunk_fwd_simt(const void* q, const void* k, const void* v, const float* log_alpha,
+                       const float* beta, const float* h0, const int32_t* cu_seqlens,
+                       int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                       void* o, float* hT, cudaStream_t stream) {
+  int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                               qkv_dtype, o, hT);
+  if (st != KDA_OK) return st;
+  return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                             qkv_dtype, o, hT, stream);
+}
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                  const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                  int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
+                  cudaStream_t stream) {
+  int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                               qkv_dtype, o, hT);
+  if (st != KDA_OK) return st;
+  return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                             qkv_dtype, o, hT, stream);
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
+                    const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_heads,
+                    kda_dtype qkv_dtype, kda_dtype gate_dtype, cudaStream_t stream) {
+  if ((qkv_dtype != KDA_F32 && qkv_dtype != KDA_BF16) ||
+      (gate_dtype != KDA_F32 && gate_dtype != KDA_BF16))
+    return KDA_ERR_DTYPE;
+  if (n_seqs <= 0 || n_heads <= 0 || (int64_t)n_seqs * n_heads > (int64_t)INT32_MAX)
+    return KDA_ERR_SHAPE;
+  if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, state, o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return KDA_ERR_ALIGN;
+  if (qkv_dtype == KDA_BF16) {
+    if (gate_dtype == KDA_BF16)
+      return launch_decode<__nv_bfloat16, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o,
+                                                         n_seqs, n_heads, stream);
+    return launch_decode<__nv_bfloat16, float>(q, k, v, log_alpha, beta, state, o, n_seqs,
+                                               n_heads, stream);
+  }
+  if (gate_dtype == KDA_BF16)
+    return launch_decode<float, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o, n_seqs,
+                                               n_heads, stream);
+  return launch_decode<float, float>(q, k, v, log_alpha, beta, state, o, n_seqs, n_heads, stream);
+}
+
+int kda_device_status(cudaStream_t stream) {
+  int h = 0;
+  if (cudaMemcpyFromSymbolAsync(&h, g_kda_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+  if (h != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_kda_device_error, &zero, sizeof(int), 0,
+                                cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+        cudaStreamSynchronize(stream) != cudaSuccess)
+      return KDA_ERR_CUDA;
+  }
+  if (h & kda::DEVERR_TIMEOUT) return KDA_ERR_TIMEOUT;
+  if (h & kda::DEVERR_SEQLENS) return KDA_ERR_SEQLENS;
+  return KDA_OK;
+}
+
+const char* kda_status_string(int status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_NULL: return "KDA_ERR_NULL: a required pointer is NULL";
+    case KDA_ERR_SHAPE: return "KDA_ERR_SHAPE: a size is out of range";
+    case KDA_ERR_DTYPE: return "KDA_ERR_DTYPE: unsupported dtype";
+    case KDA_ERR_ALIGN: return "KDA_ERR_ALIGN: a tensor pointer is not 16-byte aligned";
+    case KDA_ERR_SEQLENS: return "KDA_ERR_SEQLENS: cu_seqlens inconsistent";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call or launch failed";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    default: return "unknown kda_status";
+  }
+}
+
+}  // extern "C"

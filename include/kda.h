@@ -1,0 +1,144 @@
+/*
+ * kda.h - C ABI of the B200 (sm_100a) Kimi Delta Attention library.
+ *
+ * Kimi Delta Attention (KDA) is the channel-wise gated delta rule of Kimi Linear
+ * (Kimi Linear summary, section 3 "Kimi Delta Attention"):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * S is a per-(sequence, head) 128 x 128 fp32 state (row = key channel, column =
+ * value channel), alpha_t in (0,1]^128 is a per-channel decay passed in log
+ * space (log_alpha = log alpha <= 0), beta_t is a scalar per token and head,
+ * and q, k are expected to be L2-normalised already (section 4: queries and keys
+ * are normalised to unit length before the recurrence; this library applies no
+ * normalisation and no output scale).
+ *
+ * Two operations:
+ *   kda_chunk_fwd    prefill: the chunkwise-parallel form (chunks of 64 tokens,
+ *                    WY representation + UT transform, section 3.1
+ *                    "Hardware-Efficient Chunkwise Algorithm"), with an optional
+ *                    initial state and the final state returned (appendix C:
+ *                    chunk_kda with initial_state and chunk_size = 64).
+ *   kda_decode_step  generation: one recurrent update per (sequence, head) on a
+ *                    state held in place (section 6.3: autoregressive generation
+ *                    uses recurrent updates on a fixed 128 x 128 state).
+ *
+ * Conventions for every entry point:
+ *   - Head dimension is fixed: d_k = d_v = 128.
+ *   - Every pointer is a DEVICE pointer owned by the caller. The library
+ *     allocates no device memory and keeps no per-call state.
+ *   - Calls are asynchronous and ordered on `stream`. A return of KDA_OK means
+ *     "arguments validated and kernel launched"; device-side problems (bad
+ *     cu_seqlens contents) are reported later by kda_device_status().
+ *   - Tensor pointers must be 16-byte aligned; tensors are dense, row-major,
+ *     token-major with the strides implied by the shapes below.
+ *   - Outputs may not alias inputs (except the decode state, updated in place).
+ */
+#ifndef KDA_B200_H
+#define KDA_B200_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_NULL = -1,     /* a required pointer is NULL */
+  KDA_ERR_SHAPE = -2,    /* a size is out of range (n_heads <= 0, t_total < 0, ...) */
+  KDA_ERR_DTYPE = -3,    /* unsupported dtype enum */
+  KDA_ERR_ALIGN = -4,    /* a tensor pointer is not 16-byte aligned */
+  KDA_ERR_SEQLENS = -5,  /* cu_seqlens inconsistent (host check, or reported by the device) */
+  KDA_ERR_CUDA = -6,     /* a CUDA runtime call or kernel launch failed */
+  KDA_ERR_TIMEOUT = -7   /* a kernel gave up a bounded wait and skipped its work */
+} kda_status;
+
+/*
+ * kda_chunk_fwd - chunkwise KDA prefill over a packed batch of sequences.
+ *
+ * Computes, for every sequence n and head h, the recurrence above over the
+ * sequence's tokens starting from h0[n,h] (or zero), writes o for every token and
+ * the state after the sequence's last token to hT[n,h]. The sequence is cut into
+ * chunks of 64 tokens, restarting at each sequence's first token, so no chunk
+ * crosses a sequence boundary; the last chunk of a sequence may be shorter.
+ *
+ * Arguments:
+ *   q, k, v     [t_total, n_heads, 128], dtype qkv_dtype (KDA_F32 or KDA_BF16)
+ *   log_alpha   [t_total, n_heads, 128] fp32, entries finite and <= 0
+ *   beta        [t_total, n_heads] fp32, normally in [0, 1]
+ *   h0          [n_seqs, n_heads, 128, 128] fp32, or NULL for a zero initial state
+ *   cu_seqlens  [n_seqs + 1] int32 on the device: sequence n owns tokens
+ *               [cu_seqlens[n], cu_seqlens[n+1]); must start at 0, be
+ *               non-decreasing and end at t_total. NULL means one sequence of
+ *               t_total tokens (then n_seqs must be 1).
+ *   n_seqs, t_total, n_heads   sizes (t_total may be 0)
+ *   qkv_dtype   dtype of q, k, v and o
+ *   o           [t_total, n_heads, 128] output, dtype qkv_dtype
+ *   hT          [n_seqs, n_heads, 128, 128] fp32 output, or NULL to skip
+ *   stream      CUDA stream for the launch
+ *
+ * Precision: KDA_F32 inputs take the fp32 CUDA-core path throughout. KDA_BF16
+ * inputs take the tensor-core path (bf16 operands, fp32 accumulation, fp32 state).
+ * Device-side cu_seqlens errors are clamped to stay in bounds and flagged for
+ * kda_device_status().
+ * Returns KDA_OK or a negative kda_status.
+ */
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                  const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                  int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
+                  cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_simt - the same operation as kda_chunk_fwd, always on the fp32
+ * CUDA-core chunk kernel (exact element-wise decay factors, fp32 math). Same
+ * arguments, layouts and errors. It is the precision path for fp32 inputs and a
+ * second, independent GPU implementation of the chunk form for bf16 inputs.
+ */
+int kda_chunk_fwd_simt(const void* q, const void* k, const void* v, const float* log_alpha,
+                       const float* beta, const float* h0, const int32_t* cu_seqlens,
+                       int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                       void* o, float* hT, cudaStream_t stream);
+
+/*
+ * kda_decode_step - one recurrent KDA update per (sequence, head), in place.
+ *
+ * For each of the n_seqs * n_heads states (section 6.3 "Complexity Analysis":
+ * generation uses recurrent updates on the fixed state), with
+ * alpha = exp(log_alpha):
+ *     S' = Diag(alpha) S;  delta = beta (v - S'^T k);  S <- S' + k delta^T;
+ *     o = S^T q   (computed as S'^T q + (k^T q) delta)
+ *
+ * Arguments:
+ *   q, k, v     [n_seqs, n_heads, 128], dtype qkv_dtype
+ *   log_alpha   [n_seqs, n_heads, 128], dtype gate_dtype, entries <= 0
+ *   beta        [n_seqs, n_heads], dtype gate_dtype
+ *   state       [n_seqs, n_heads, 128, 128] fp32, read and overwritten in place
+ *   o           [n_seqs, n_heads, 128] output, dtype qkv_dtype
+ *   qkv_dtype, gate_dtype   KDA_F32 or KDA_BF16 each
+ * Returns KDA_OK or a negative kda_status.
+ */
+int kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
+                    const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_heads,
+                    kda_dtype qkv_dtype, kda_dtype gate_dtype, cudaStream_t stream);
+
+/*
+ * kda_device_status - read and clear the library's device-side error word.
+ * Synchronises `stream`. Returns KDA_OK, KDA_ERR_SEQLENS (a kernel saw
+ * cu_seqlens that were not monotone or ran past t_total, and clamped them),
+ * KDA_ERR_TIMEOUT (a kernel gave up a bounded wait), or KDA_ERR_CUDA.
+ */
+int kda_device_status(cudaStream_t stream);
+
+/* kda_status_string - a static, human-readable name for a kda_status value. */
+const char* kda_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_H */

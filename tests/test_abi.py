@@ -1,0 +1,90 @@
+"""The C-ABI library loads, exports every declared entry point, and validates
+arguments on the host (no GPU needed: every case here returns before any CUDA
+call)."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from channel_wise_gated_b200 import _native, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(kda_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _native.load()
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("kda_chunk_fwd", "kda_chunk_fwd_simt", "kda_decode_step", "kda_device_status",
+              "kda_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in kda.h but not exported"
+        assert name in _native.SIGNATURES, f"{name} has no binding signature"
+
+
+def test_status_strings(lib):
+    for st in range(0, -8, -1):
+        s = _native.status_string(st)
+        assert s.startswith("KDA_")
+    assert "unknown" in _native.status_string(-99)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every case fails validation first
+
+
+def _chunk(lib, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, h0=None, cu=None, n=1, T=64, H=2,
+                dt=_native.KDA_BF16, o=FAKE, hT=None, stream=None)
+    args.update(over)
+    return lib.kda_chunk_fwd(args["q"], args["k"], args["v"], args["la"], args["b"], args["h0"],
+                             args["cu"], args["n"], args["T"], args["H"], args["dt"], args["o"],
+                             args["hT"], args["stream"])
+
+
+def test_chunk_validation(lib):
+    assert _chunk(lib, q=None) == _native.KDA_ERR_NULL
+    assert _chunk(lib, o=None) == _native.KDA_ERR_NULL
+    assert _chunk(lib, H=0) == _native.KDA_ERR_SHAPE
+    assert _chunk(lib, T=-1) == _native.KDA_ERR_SHAPE
+    assert _chunk(lib, n=0) == _native.KDA_ERR_SHAPE
+    assert _chunk(lib, dt=7) == _native.KDA_ERR_DTYPE
+    assert _chunk(lib, k=FAKE + 8) == _native.KDA_ERR_ALIGN
+    assert _chunk(lib, hT=FAKE + 4) == _native.KDA_ERR_ALIGN
+    assert _chunk(lib, n=2, cu=None) == _native.KDA_ERR_SEQLENS
+    assert lib.kda_chunk_fwd_simt(None, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2,
+                                  _native.KDA_F32, FAKE, None, None) == _native.KDA_ERR_NULL
+
+
+def test_decode_validation(lib):
+    f = lib.kda_decode_step
+    bf = _native.KDA_BF16
+    assert f(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, bf, bf, None) == _native.KDA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 2, bf, bf, None) == _native.KDA_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, bf, bf, None) == _native.KDA_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 3, bf, None) == _native.KDA_ERR_DTYPE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE, 4, 2, bf, bf, None) == _native.KDA_ERR_ALIGN
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_native, "_lib", None)
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        _native.load(str(tmp_path / "missing.so"))

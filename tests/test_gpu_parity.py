@@ -1,0 +1,244 @@
+"""GPU parity: the CUDA kernels (through the C ABI) against the fp64 oracle.
+
+Error metric (global, as the tolerance is stated): max|x - x_ref| / max|x_ref|
+over the whole compared tensor. Bounds: 1e-4 for fp32 inputs, 2e-2 for bf16
+inputs with an fp32 state, for both o and the final state.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import kda_inputs
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+def rel_err(x, ref):
+    x = x.detach().double().cpu().numpy() if isinstance(x, torch.Tensor) else np.asarray(x)
+    ref = np.asarray(ref)
+    den = np.abs(ref).max()
+    return float(np.abs(x - ref).max() / (den if den > 0 else 1.0))
+
+
+@pytest.fixture(scope="module")
+def kda():
+    from channel_wise_gated_b200 import build
+    build.build()
+    import channel_wise_gated_b200 as m
+    return m
+
+
+def _oracle(inp, heads=None):
+    sel = (lambda t: t[:, heads]) if heads is not None else (lambda t: t)
+    h0 = inp["h0"]
+    if h0 is not None and heads is not None:
+        h0 = h0[:, heads]
+    return oracle.oracle_forward(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]),
+                                 sel(inp["log_alpha"]), sel(inp["beta"]), h0=h0,
+                                 cu_seqlens=inp["cu_seqlens"].cpu(), col_block=16)
+
+
+def _run(kda, inp, kernel="auto"):
+    return kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                         h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], kernel=kernel)
+
+
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_config0_tiny_fp32(kda, kernel):
+    inp = kda_inputs.make_config(0, device="cuda")
+    o, hT = _run(kda, inp, kernel)
+    o_ref, h_ref = _oracle(inp)
+    assert rel_err(o, o_ref) <= TOL_F32
+    assert rel_err(hT, h_ref) <= TOL_F32
+    assert kda.device_status() == 0
+
+
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_config1_prefill_bf16(kda, kernel):
+    inp = kda_inputs.make_config(1, device="cuda")
+    o, hT = _run(kda, inp, kernel)
+    o_ref, h_ref = _oracle(inp)
+    e_o, e_s = rel_err(o, o_ref), rel_err(hT, h_ref)
+    print(f"config1 {kernel}: o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+
+
+def test_config2_varlen(kda):
+    inp = kda_inputs.make_config(2, device="cuda")
+    assert len(inp["lens"]) == 16
+    o, hT = _run(kda, inp)
+    heads = [0, 13, 31]   # sampled heads, every sequence, every token
+    o_ref, h_ref = _oracle(inp, heads)
+    e_o = rel_err(o[:, heads], o_ref)
+    e_s = rel_err(hT[:, heads], h_ref)
+    print(f"config2: o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+    assert kda.device_status() == 0
+
+
+def test_config3_long_context(kda):
+    """Full 1,048,576-token launch; the oracle follows 2 sampled heads end to end."""
+    inp = kda_inputs.make_config(3, device="cuda")
+    o, hT = _run(kda, inp)
+    heads = [5, 26]
+    o_ref, h_ref = _oracle(inp, heads)
+    e_o = rel_err(o[:, heads], o_ref)
+    e_s = rel_err(hT[:, heads], h_ref)
+    print(f"config3: o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+    # the tail of the sequence separately (errors must not grow along the sequence)
+    assert rel_err(o[-4096:, heads], o_ref[-4096:]) <= TOL_BF16
+    del inp, o, hT
+    torch.cuda.empty_cache()
+
+
+def test_config4_decode(kda):
+    """1000 in-place decode steps for all 8,192 states; oracle on 64 sampled chains."""
+    c = kda_inputs.DECODE_CONFIG
+    inp = kda_inputs.make_decode_config(device="cuda")
+    state = inp["state"].clone()
+    outs = []
+    for s in range(c.steps):
+        outs.append(kda.decode_step(inp["q"][s], inp["k"][s], inp["v"][s],
+                                    inp["log_alpha"][s], inp["beta"][s], state))
+    o = torch.stack(outs)
+    g = torch.Generator().manual_seed(44)
+    flat = torch.randperm(c.n_seqs * c.n_heads, generator=g)[:64]
+    seqs, heads = (flat // c.n_heads).tolist(), (flat % c.n_heads).tolist()
+    pick = lambda t: torch.stack([t[:, n, h] for n, h in zip(seqs, heads)], dim=1)[:, :, None]
+    st0 = torch.stack([inp["state"][n, h] for n, h in zip(seqs, heads)])[:, None]
+    o_ref, s_ref = oracle.oracle_decode_steps(pick(inp["q"]), pick(inp["k"]), pick(inp["v"]),
+                                              pick(inp["log_alpha"]), pick(inp["beta"]), st0,
+                                              col_block=32)
+    o_gpu = torch.stack([o[:, n, h] for n, h in zip(seqs, heads)], dim=1)[:, :, None]
+    s_gpu = torch.stack([state[n, h] for n, h in zip(seqs, heads)])[:, None]
+    e_o, e_s = rel_err(o_gpu, o_ref), rel_err(s_gpu, s_ref)
+    print(f"config4: o {e_o:.2e} state {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+
+
+def test_decode_fp32_exact(kda):
+    inp = kda_inputs.make_decode(3, 4, 20, torch.float32, torch.float32, seed=9, device="cuda")
+    state = inp["state"].clone()
+    o = torch.stack([kda.decode_step(inp["q"][s], inp["k"][s], inp["v"][s], inp["log_alpha"][s],
+                                     inp["beta"][s], state) for s in range(20)])
+    o_ref, s_ref = oracle.oracle_decode_steps(inp["q"], inp["k"], inp["v"], inp["log_alpha"],
+                                              inp["beta"], inp["state"])
+    assert rel_err(o, o_ref) <= TOL_F32
+    assert rel_err(state, s_ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_ragged_lengths(kda, T, dtype):
+    inp = kda_inputs.make_prefill([T], 3, dtype, torch.float32, 3.0, True, seed=T, device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    assert rel_err(o, o_ref) <= tol
+    assert rel_err(hT, h_ref) <= tol
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_varlen_with_empty_and_tiny_sequences(kda, dtype):
+    lens = [0, 1, 130, 0, 64, 7]
+    inp = kda_inputs.make_prefill(lens, 2, dtype, torch.float32, 3.0, True, seed=21, device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    assert rel_err(o, o_ref) <= tol
+    assert rel_err(hT, h_ref) <= tol
+    # an empty sequence returns its initial state unchanged
+    assert torch.equal(hT[0], inp["h0"][0]) and torch.equal(hT[3], inp["h0"][3])
+    assert kda.device_status() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_strong_decay_stress(kda, dtype):
+    """log alpha around -5 per token: chunk decay spans hundreds of nats."""
+    inp = kda_inputs.make_prefill([300], 2, dtype, torch.float32, -5.0, True, seed=31,
+                                  device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    assert rel_err(o, o_ref) <= tol
+    assert rel_err(hT, h_ref) <= max(tol, 1e-30)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_no_decay_full_erase(kda, dtype):
+    """alpha = 1 (log alpha = 0) and beta = 1: pure DeltaNet with full erase strength."""
+    inp = kda_inputs.make_prefill([192], 2, dtype, torch.float32, 3.0, False, seed=41,
+                                  device="cuda")
+    inp["log_alpha"].zero_()
+    inp["beta"].fill_(1.0)
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+    assert rel_err(o, o_ref) <= tol
+    assert rel_err(hT, h_ref) <= tol
+
+
+def test_zero_tokens_and_optional_outputs(kda):
+    inp = kda_inputs.make_prefill([0], 2, torch.bfloat16, torch.float32, 3.0, True, seed=1,
+                                  device="cuda")
+    o, hT = _run(kda, inp)
+    assert o.shape[0] == 0 and torch.equal(hT, inp["h0"])
+    inp = kda_inputs.make_prefill([100], 2, torch.bfloat16, torch.float32, 3.0, False, seed=2,
+                                  device="cuda")
+    o1, _ = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                          output_final_state=False)
+    o2, _ = _run(kda, inp)
+    assert torch.equal(o1, o2)
+
+
+def test_chunk_equals_decode_iterated(kda):
+    """Chunkwise prefill and the recurrent step agree on the same inputs."""
+    N, H, T = 2, 4, 150
+    inp = kda_inputs.make_prefill([T] * N, H, torch.bfloat16, torch.float32, 3.0, True, seed=51,
+                                  device="cuda")
+    o_chunk, h_chunk = _run(kda, inp)
+    state = inp["h0"].clone()
+    o_dec = torch.empty_like(o_chunk)
+    for t in range(T):
+        idx = torch.tensor([t, T + t], device="cuda")
+        o_dec[idx] = kda.decode_step(inp["q"][idx], inp["k"][idx], inp["v"][idx],
+                                     inp["log_alpha"][idx].contiguous(),
+                                     inp["beta"][idx].contiguous(), state)
+    o_ref, h_ref = _oracle(inp)
+    assert rel_err(o_chunk, o_dec.double().cpu().numpy()) <= TOL_BF16
+    assert rel_err(h_chunk, state.double().cpu().numpy()) <= TOL_BF16
+    assert rel_err(o_dec, o_ref) <= TOL_BF16
+
+
+def test_prefill_then_decode_resumes(kda):
+    """Checkpoint/resume: prefill(T) then one decode step equals prefill(T+1)."""
+    T, H = 129, 3
+    inp = kda_inputs.make_prefill([T + 1], H, torch.float32, torch.float32, 3.0, True, seed=61,
+                                  device="cuda")
+    sl = lambda t, a, b: t[a:b].contiguous()
+    _, hT = kda.chunk_fwd(sl(inp["q"], 0, T), sl(inp["k"], 0, T), sl(inp["v"], 0, T),
+                          sl(inp["log_alpha"], 0, T), sl(inp["beta"], 0, T), h0=inp["h0"])
+    state = hT[0:1].clone()
+    o_last = kda.decode_step(sl(inp["q"], T, T + 1), sl(inp["k"], T, T + 1),
+                             sl(inp["v"], T, T + 1), sl(inp["log_alpha"], T, T + 1),
+                             sl(inp["beta"], T, T + 1), state)
+    o_full, h_full = _run(kda, inp)
+    assert rel_err(o_last, o_full[T:T + 1].double().cpu().numpy()) <= TOL_F32
+    assert rel_err(state, h_full.double().cpu().numpy()) <= TOL_F32
+
+
+def test_bad_seqlens_are_clamped_and_reported(kda):
+    inp = kda_inputs.make_prefill([100, 100], 2, torch.bfloat16, torch.float32, 3.0, False,
+                                  seed=71, device="cuda")
+    cu = torch.tensor([0, 150, 120], dtype=torch.int32, device="cuda")   # not monotone
+    kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], cu_seqlens=cu)
+    assert kda.device_status() == kda._native.KDA_ERR_SEQLENS
+    assert kda.device_status() == 0   # read clears it

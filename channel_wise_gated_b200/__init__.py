@@ -20,8 +20,8 @@ from ._native import KdaError  # noqa: F401
 
 D = 128
 
-# Arithmetic type of the prefill path's contractions for bf16 inputs.
-PREFILL_COMPUTE_DTYPE = "f32"
+# Arithmetic type of the prefill contractions for bf16 inputs (bf16 operands, fp32 accumulation).
+PREFILL_COMPUTE_DTYPE = "bf16"
 
 _DT = {torch.float32: _native.KDA_F32, torch.bfloat16: _native.KDA_BF16}
 

@@ -2,11 +2,15 @@
 // stream-ordered kernel launches. All device code lives in the included headers;
 // this file is the library's single translation unit.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/kda.h"
 #include "kda_chunk_simt.cuh"
+#include "kda_chunk_tc.cuh"
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
 
@@ -61,6 +65,75 @@ int chunk_simt_dispatch(const void* q, const void* k, const void* v, const float
                                           t_total, n_heads, o, hT, stream);
 }
 
+// ---- tensor-core chunk kernel: TMA descriptors and launch ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn tensor_map_encoder() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D view [rows][cols] of a token-major tensor, box [box_r][box_c].
+bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t cols,
+               uint64_t rows, uint64_t elem_bytes, uint32_t box_c, uint32_t box_r,
+               CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem_bytes};
+  const cuuint32_t box[2] = {box_c, box_r};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
+                    const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                    int64_t t_total, int32_t n_heads, void* o, float* hT, cudaStream_t stream) {
+  using namespace kda::tc;
+  const uint64_t cols = (uint64_t)n_heads * kda::D;
+  const uint64_t rows = (uint64_t)t_total;
+  CUtensorMap mk, mq, mv, mla;
+  if (!encode_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, cols, rows, 2, 64, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, cols, rows, 2, 64, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, cols, rows, 2, DV, 64,
+                 CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, log_alpha, cols, rows, 4, 128, 64,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return KDA_ERR_CUDA;
+  if (cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)SMEM_BYTES) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  Args a;
+  a.log_alpha = log_alpha;
+  a.beta = beta;
+  a.h0 = h0;
+  a.cu_seqlens = cu_seqlens;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.hT = hT;
+  a.n_seqs = n_seqs;
+  a.n_heads = n_heads;
+  a.t_total = t_total;
+  const int64_t grid = (int64_t)n_seqs * n_heads * NSPLIT;
+  kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, a);
+  return launch_status();
+}
+
 template <typename TQ, typename TG>
 int launch_decode(const void* q, const void* k, const void* v, const void* log_alpha,
                   const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_heads,
@@ -94,6 +167,12 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_
   int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                                qkv_dtype, o, hT);
   if (st != KDA_OK) return st;
+  // bf16 inputs run on the tensor-core kernel; its TMA boxes span 64 tokens, so
+  // inputs shorter than one chunk (and fp32 inputs) take the CUDA-core kernel.
+  if (qkv_dtype == KDA_BF16 && t_total >= kda::CHUNK && t_total < (int64_t)INT32_MAX - 4 * kda::CHUNK &&
+      (int64_t)n_seqs * n_heads * kda::tc::NSPLIT < (int64_t)INT32_MAX)
+    return launch_chunk_tc(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads, o,
+                           hT, stream);
   return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                              qkv_dtype, o, hT, stream);
 }

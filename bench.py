@@ -33,6 +33,7 @@ import torch  # noqa: E402
 import kda_inputs  # noqa: E402
 
 METRIC = "KDA prefill tokens/s (H=32,d=128) & decode-step HBM GB/s vs peak, 1xB200"
+WORKLOADS = {"longctx": 3, "prefill4k": 1, "varlen16": 2}
 D = 128
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * D + 4 * D + 4 + 2 * D   # q,k,v bf16 + log_alpha f32 + beta + o
 STATE_BYTES = 4 * D * D
@@ -311,6 +312,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="longctx",
+                    choices=sorted(WORKLOADS),
+                    help="prefill workload (the headline is longctx; prefill4k is the small "
+                         "case used for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -324,7 +329,7 @@ def main():
     hbm_peak, bf16_peak, peak_kind = _peaks()
 
     # ---- prefill workload (each rank its own batch)
-    cfg = kda_inputs.PREFILL_CONFIGS[3]
+    cfg = kda_inputs.PREFILL_CONFIGS[WORKLOADS[args.workload]]
     lens = kda_inputs.config_lengths(cfg)
     inp = kda_inputs.make_prefill(lens, cfg.n_heads, cfg.qkv_dtype, torch.float32, cfg.x_mean,
                                   cfg.h0, cfg.seed + 100 * rank, "cuda")

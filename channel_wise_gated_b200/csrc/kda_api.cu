@@ -44,11 +44,11 @@ int launch_chunk_simt(const void* q, const void* k, const void* v, const float* 
                       int32_t n_seqs, int64_t t_total, int32_t n_heads, void* o, float* hT,
                       cudaStream_t stream) {
   const size_t smem = sizeof(kda::SimtSmem);
-  if (cudaFuncSetAttribute(kda::chunk_simt_kernel<TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(kda::kda_chunk_simt_kernel<TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return KDA_ERR_CUDA;
   dim3 grid((unsigned)(n_seqs * n_heads), kda::D / kda::SIMT_DV);
-  kda::chunk_simt_kernel<TQ><<<grid, kda::SIMT_THREADS, smem, stream>>>(
+  kda::kda_chunk_simt_kernel<TQ><<<grid, kda::SIMT_THREADS, smem, stream>>>(
       static_cast<const TQ*>(q), static_cast<const TQ*>(k), static_cast<const TQ*>(v), log_alpha,
       beta, h0, cu_seqlens, n_seqs, t_total, n_heads, static_cast<TQ*>(o), hT);
   return launch_status();
@@ -139,7 +139,7 @@ int launch_decode(const void* q, const void* k, const void* v, const void* log_a
                   const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_heads,
                   cudaStream_t stream) {
   const unsigned chains = (unsigned)n_seqs * (unsigned)n_heads;
-  kda::decode_step_kernel<TQ, TG><<<chains, kda::DEC_THREADS, 0, stream>>>(
+  kda::kda_decode_step_kernel<TQ, TG><<<chains, kda::DEC_THREADS, 0, stream>>>(
       static_cast<const TQ*>(q), static_cast<const TQ*>(k), static_cast<const TQ*>(v),
       static_cast<const TG*>(log_alpha), static_cast<const TG*>(beta), state, static_cast<TQ*>(o));
   return launch_status();

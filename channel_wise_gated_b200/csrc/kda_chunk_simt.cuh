@@ -49,7 +49,7 @@ struct SimtSmem {
 
 template <typename TQ>
 __global__ void __launch_bounds__(SIMT_THREADS, 1)
-chunk_simt_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const TQ* __restrict__ v,
+kda_chunk_simt_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const TQ* __restrict__ v,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
                   const float* __restrict__ h0, const int32_t* __restrict__ cu_seqlens,
                   int n_seqs, int64_t t_total, int n_heads, TQ* __restrict__ o,

@@ -26,7 +26,7 @@ constexpr int DEC_ROWS_PER_WARP = D / (DEC_THREADS / 32);  // 16
 
 template <typename TQ, typename TG>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
-decode_step_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const TQ* __restrict__ v,
+kda_decode_step_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const TQ* __restrict__ v,
                    const TG* __restrict__ log_alpha, const TG* __restrict__ beta,
                    float* __restrict__ state, TQ* __restrict__ o) {
   const int chain = blockIdx.x;          // (sequence, head) flattened

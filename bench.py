@@ -127,10 +127,15 @@ def _barrier(ws):
         torch.distributed.barrier()
 
 
+def _reduce_device() -> str:
+    # NCCL reduces device tensors; gloo (the CPU test backend) host tensors
+    return "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+
+
 def _max_over_ranks(x: float, ws: int) -> float:
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -138,9 +143,19 @@ def _max_over_ranks(x: float, ws: int) -> float:
 def _sum_over_ranks(x: float, ws: int) -> float:
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_reduce_device())
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
     return float(t.item())
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch (replicas): seeds are distinct per rank."""
+    return base_seed + 100 * rank
+
+
+def replica_throughput(units: float, ms: float, ws: int) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return _sum_over_ranks(units, ws) / (_max_over_ranks(ms, ws) / 1e3)
 
 
 def _oracle_sample_rate(cfg_idx: int, target_s: float, seed_heads=(0, 1), max_tokens=1 << 20):
@@ -332,7 +347,7 @@ def main():
     cfg = kda_inputs.PREFILL_CONFIGS[WORKLOADS[args.workload]]
     lens = kda_inputs.config_lengths(cfg)
     inp = kda_inputs.make_prefill(lens, cfg.n_heads, cfg.qkv_dtype, torch.float32, cfg.x_mean,
-                                  cfg.h0, cfg.seed + 100 * rank, "cuda")
+                                  cfg.h0, replica_seed(cfg.seed, rank), "cuda")
     T, H = sum(lens), cfg.n_heads
     N = len(lens)
     inp["o"] = torch.empty_like(inp["q"])
@@ -344,8 +359,7 @@ def main():
         total_ms, per_launch = time_prefill(kda, inp, args.steps, args.warmup, ws, stream)
     clocks = clk.summary()
     max_ms = _max_over_ranks(total_ms, ws)
-    tokens_all = _sum_over_ranks(float(T * args.steps), ws)
-    value = tokens_all / (max_ms / 1e3)
+    value = replica_throughput(float(T * args.steps), total_ms, ws)
     avg_launch_ms = sum(per_launch) / len(per_launch)
     achieved = step_bytes / (avg_launch_ms / 1e3) / 1e9
 
@@ -353,11 +367,15 @@ def main():
     dcfg = kda_inputs.DECODE_CONFIG
     n_pool = 50   # distinct per-step inputs cycled through (all > L2 with the state)
     dec = kda_inputs.make_decode(dcfg.n_seqs, dcfg.n_heads, n_pool, dcfg.qkv_dtype,
-                                 dcfg.gate_dtype, dcfg.x_mean, dcfg.state_std, dcfg.seed, "cuda")
-    dec_ms = time_decode(kda, dec, args.decode_steps, args.warmup, stream)
+                                 dcfg.gate_dtype, dcfg.x_mean, dcfg.state_std,
+                                 replica_seed(dcfg.seed, rank), "cuda")
+    _barrier(ws)
+    dec_ms = _max_over_ranks(time_decode(kda, dec, args.decode_steps, args.warmup, stream), ws)
     chains = dcfg.n_seqs * dcfg.n_heads
     dec_step_us = dec_ms / args.decode_steps * 1e3
-    dec_gbs = chains * DECODE_BYTES_PER_CHAIN / (dec_step_us / 1e6) / 1e9
+    # whole-job bytes per step (every replica moves its own states) over the slowest rank
+    dec_gbs = replica_throughput(float(chains * DECODE_BYTES_PER_CHAIN * args.decode_steps),
+                                 dec_ms, ws) / 1e9
     del dec
     torch.cuda.empty_cache()
 
@@ -365,9 +383,8 @@ def main():
     e2e = None
     if not args.no_e2e:
         ms, h2d, d2h = time_e2e(kda, inp, args.e2e_steps, stream)
-        ms = _max_over_ranks(ms, ws)
-        e2e_tokens = _sum_over_ranks(float(T * args.e2e_steps), ws)
-        e2e = {"value": e2e_tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": replica_throughput(float(T * args.e2e_steps), ms, ws),
+               "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
     cpu = None
@@ -398,7 +415,7 @@ def main():
             "decode": {"workload": dcfg.name, "steps": args.decode_steps,
                        "us_per_step": dec_step_us, "GBps": dec_gbs,
                        "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak,
-                                    "unit": "GB/s", "frac": dec_gbs / hbm_peak,
+                                    "unit": "GB/s", "frac": dec_gbs / (hbm_peak * ws),
                                     "algorithmic_bytes_per_step": chains * DECODE_BYTES_PER_CHAIN},
                        "gpu_launches": args.decode_steps,
                        "l2": "state 512 MiB > L2"},

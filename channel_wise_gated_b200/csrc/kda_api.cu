@@ -111,8 +111,8 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, cols, rows, 2, DV, 64,
-                 CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !encode_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, cols, rows, 2, 64, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, log_alpha, cols, rows, 4, 128, 64,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return KDA_ERR_CUDA;
@@ -129,7 +129,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.n_seqs = n_seqs;
   a.n_heads = n_heads;
   a.t_total = t_total;
-  const int64_t grid = (int64_t)n_seqs * n_heads * NSPLIT;
+  const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
   kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, a);
   return launch_status();
 }
@@ -170,7 +170,7 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_
   // bf16 inputs run on the tensor-core kernel; its TMA boxes span 64 tokens, so
   // inputs shorter than one chunk (and fp32 inputs) take the CUDA-core kernel.
   if (qkv_dtype == KDA_BF16 && t_total >= kda::CHUNK && t_total < (int64_t)INT32_MAX - 4 * kda::CHUNK &&
-      (int64_t)n_seqs * n_heads * kda::tc::NSPLIT < (int64_t)INT32_MAX)
+      (int64_t)n_seqs * n_heads < (int64_t)INT32_MAX)
     return launch_chunk_tc(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads, o,
                            hT, stream);
   return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,

@@ -9,37 +9,44 @@
 //   Delta = T diag(beta) V - T diag(beta) (K * e^G) S
 //   O = (Q * e^G) S + P Delta,     S <- Diag(e^{G_C}) S + (K * e^{G_C - G})^T Delta
 //
-// Decay factors. One reference row m (the chunk's middle row) splits every pairwise
-// factor as e^{G_r - G_i} = E_r * F_i with E = e^{G - G_m}, F = e^{G_m - G} = 1/E, so
-// the two Gram matrices A and P are one tensor-core product [K*E ; Q*E] (K*F)^T.
-// The remaining factors fold into the operands:
-//   K * e^G = (K * E) Diag(e^{G_m}),  Q * e^G = (Q * E) Diag(e^{G_m}),
-//   K * e^{G_C - G} = (K * F) Diag(e^{G_C - G_m}),
-// so only three bf16 tiles per chunk are built: Rk = K*E, Rq = Q*E, Ck = K*F, and
-//   S' = Diag(e^{G_m}) S          (the bf16 state operand)
+// Decay factors. The chunk's last row is the reference: with E = e^{G - G_C} (>= 1)
+// and its reciprocal F = e^{G_C - G} (<= 1), every pairwise factor is
+// e^{G_r - G_i} = E_r F_i, so A and P come out of one tensor-core product
+// [K*E ; Q*E] (K*F)^T, and the remaining factors fold into the state operand:
+//   Rk = K*E, Rq = Q*E, Ck = K*F           (three bf16 tiles per chunk)
+//   S'' = Diag(e^{G_C}) S                  (the decayed state, the bf16 MMA operand)
 //   W' = T diag(beta) Rk,  U = T diag(beta) V
-//   Delta = U - W' S',  O = Rq S' + P Delta
-//   S <- Diag(e^{G_C}) S + Diag(e^{G_C - G_m}) Ck^T Delta
-// Delta and Rq S' come out of ONE 128-row MMA: A = [-W' ; Rq] accumulating onto
-// [U ; 0]; O += P Delta then accumulates onto the Rq S' rows. (The tensor pipe
-// costs about the same per instruction for any N <= 128, so stacking saves time.)
-// This is exact in real arithmetic. It needs E and F inside the floating-point
-// range, so a chunk whose decay range max_c (G_0c - G_63c) exceeds 60 nats takes an
-// exact path instead (the pages' reason for secondary chunking): pairwise factors
-// evaluated element by element for A and P, and tiles built with reference row
-// "before the chunk" (E = e^G, Ck = K * e^{G_C - G}, all factors <= 1).
+//   Delta = U - W' S'',  O = Rq S'' + P Delta,  S <- S'' + Ck^T Delta
+// so the state update is a plain accumulate onto the decayed fp32 state. This is
+// exact in real arithmetic. E must stay in range: a chunk whose decay range
+// max_c (G_0c - G_63c) exceeds 60 nats takes an exact path instead (the pages'
+// reason for secondary chunking): A and P from pairwise factors evaluated element
+// by element, Rk and Rq built about the point before the chunk (K e^G, Q e^G, all
+// factors <= 1) and the undecayed state as the operand.
 //
-// Partition. Columns of S evolve independently, so a CTA owns one (sequence, head)
-// and DV = 32 value columns: 4 CTAs per head. Per CTA (608 threads), a pipeline
-// three chunks deep:
-//   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars
-//   warps 8-11  prep B (chunk c+1): Gram readout, UT solve, T*beta tile, W' tile
-//   warps 12-15 state  (chunk c):   Delta tile, fp32 state update, S' tile, output
-//   warp 16     TMA producer (k, q, v tiles; L2 prefetch of the log-decay)
-//   warp 17     tcgen05.mma issuer for the sequential state pass; TMEM owner
-//   warp 18     tcgen05.mma issuer for prep (Gram, W', U)
-// Every wait is bounded; a timeout flags KDA_ERR_TIMEOUT and all roles leave
-// their loops.
+// Layout. One CTA owns one (sequence, head) and all 128 value columns. The state
+// lives in tensor memory for the whole sequence, transposed (lane = value column,
+// column = key channel), so every state product has the state as its A operand:
+//   [O | Delta]^T = S''^T [Rq ; -W']^T   (A = S''^T read from TMEM, M=128, N=128)
+//   S^T += Delta^T Ck,  O^T += Delta^T P^T,  U^T = V^T (T beta)^T
+//   W'^T = -Rk^T (T beta)^T               (the -W' tile is written from it)
+// TMEM (512 columns):   0 S^T fp32 | 128 S''^T bf16 pairs | 192 O (odd chunks) |
+//   256 U then Delta | 320 O (even chunks) | 384 Gram [A;P] | 448 -W'^T
+// The stacked B operand alternates [-W' ; Rq] (even chunks) and [Rq ; -W'] (odd)
+// so that Delta always lands in columns 256-319 while the output alternates
+// between the two regions around it: the output of chunk c is read while chunk
+// c+1 is already accumulating.
+//
+// Roles (640 threads), a pipeline three chunks deep:
+//   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars;
+//               its first thread issues the k/q TMA loads and the L2 prefetch of the
+//               log-decay
+//   warps 8-11  prep B (chunk c+1): Gram readout, UT solve, T*beta tile, W' tile;
+//               its first thread issues the Gram and W' products
+//   warps 12-19 state  (chunk c):   decay S in TMEM and write S'', Delta tile, output;
+//               its first thread issues the state products, U and the v TMA loads
+// Every mbarrier wait is bounded; a timeout flags KDA_ERR_TIMEOUT and every role
+// leaves (a group keeps meeting at its own named barriers, doing no work).
 #pragma once
 
 #include "kda_common.cuh"
@@ -50,78 +57,84 @@ namespace tc {
 
 using namespace sm100;
 
-constexpr int DV = 32;
-constexpr int NSPLIT = D / DV;
 constexpr int PA_WARPS = 8;
 constexpr int PB_WARP0 = 8;
 constexpr int ST_WARP0 = 12;
-constexpr int LD_WARP = 16;
-constexpr int MC_WARP = 17;
-constexpr int MP_WARP = 18;
-constexpr int THREADS = 19 * 32;
+constexpr int ST_WARPS = 8;
+constexpr int THREADS = 20 * 32;
 constexpr int PA_THREADS = PA_WARPS * 32;
 constexpr int PB_THREADS = 128;
-constexpr int ST_THREADS = 128;
+constexpr int ST_THREADS = ST_WARPS * 32;
+static_assert(PB_WARP0 % 4 == 0 && ST_WARP0 % 4 == 0, "TMEM lane quarters follow warp % 4");
 constexpr uint32_t BAR_PA = 1, BAR_PB = 2, BAR_ST = 3;   // named barriers (0 is __syncthreads)
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float GUARD_LOG2 = 60.0f * 1.4426950408889634f;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 
 // ---- shared memory layout (offsets from a 1024-byte aligned base) ----
-constexpr uint32_t QR_BYTES = 32768;     // [Rk/W' rows 0-63 ; Rq rows 64-127], 2 kblocks x 16 KB
-constexpr uint32_t CKP_BYTES = 24576;    // Ck [64][128] (16 KB) | P [64][64] (8 KB)
-constexpr uint32_t V_BYTES = 4096;       // [64][32] bf16, 64B swizzle
-constexpr uint32_t OFF_QR = 0;
-constexpr uint32_t OFF_CKP = OFF_QR + 3 * QR_BYTES;
-constexpr uint32_t OFF_V = OFF_CKP + 2 * CKP_BYTES;
-constexpr uint32_t OFF_SP = OFF_V + 3 * V_BYTES;      // S' [128][32] bf16, 64B swizzle
-constexpr uint32_t OFF_DL = OFF_SP + 8192;            // Delta [64][32] bf16, 64B swizzle
-// prep B workspace (also the staging area of the exact path, >= 32 KB contiguous)
-constexpr uint32_t OFF_TB = OFF_DL + 4096;            // [T*beta ; 0] [128][64] bf16, 128B swizzle
+// Stage tile: 2 kblocks (channels 0-63, 64-127) x [128 rows][128 B], 128B swizzle.
+// Rows 0-63 / 64-127 hold k (then Rk, then -W') and q (then Rq): k on top for even
+// chunks, q on top for odd chunks.
+constexpr uint32_t KQ_BYTES = 32768;
+constexpr uint32_t CKP_BYTES = 24576;    // Ck [2 kblocks][64][128 B] (16 KB) | P [64][128 B] (8 KB)
+constexpr uint32_t OFF_KQ = 0;
+constexpr uint32_t OFF_CKP = OFF_KQ + 3 * KQ_BYTES;
+constexpr uint32_t OFF_V = OFF_CKP + 2 * CKP_BYTES;   // v [2 column blocks][64][128 B]
+constexpr uint32_t OFF_TB = OFF_V + 16384;            // T*beta [64 r][64 i] bf16, K-major
+constexpr uint32_t OFF_DT = OFF_TB + 8192;            // Delta^T [128 j][64 r] bf16, K-major
 constexpr int AW = 68;                                // fp32 pitch of the A / T workspace
-constexpr uint32_t OFF_AW = OFF_TB + 16384;
+constexpr uint32_t OFF_AW = OFF_DT + 16384;           // also the exact path's staging area
 constexpr uint32_t OFF_XS = OFF_AW + 64 * AW * 4;     // 6 extra 16x16 fp32 blocks
 constexpr uint32_t OFF_SCR = OFF_XS + 6 * 1024;       // 4 per-warp 16x16 scratch blocks
 constexpr uint32_t OFF_BETA = OFF_SCR + 4 * 1024;     // [3][64]
-constexpr uint32_t OFF_SCAL = OFF_BETA + 3 * 64 * 4;  // [3 slots][3][128]: e^{G_m}, e^{G_C}, e^{G_C-G_m}
-constexpr uint32_t OFF_WSUM = OFF_SCAL + 9 * 128 * 4; // [8][128] cumsum warp totals
-constexpr uint32_t OFF_GROW = OFF_WSUM + 8 * 128 * 4; // [3][128] G2 of rows 0, 31, 63
-constexpr uint32_t OFF_XFLAG = OFF_GROW + 3 * 128 * 4; // [3] exact-path flag per slot
+constexpr uint32_t OFF_SCAL = OFF_BETA + 3 * 64 * 4;  // [3 slots][2][128]: state decay, operand scale
+constexpr uint32_t OFF_WSUM = OFF_SCAL + 6 * 128 * 4; // [8][128] cumsum warp totals
+constexpr uint32_t OFF_GROW = OFF_WSUM + 8 * 128 * 4; // [2][128] G of rows 0 and 63 (log2 units)
+constexpr uint32_t OFF_XFLAG = OFF_GROW + 2 * 128 * 4; // [3] exact-path flag per slot
 constexpr uint32_t OFF_BAR = OFF_XFLAG + 16;
-constexpr int NBARS = 40;
+constexpr int NBARS = 32;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr uint32_t SMEM_USED = OFF_MISC + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_SCR + 4 * 1024 - OFF_TB >= 32768, "exact-path staging needs 32 KB");
+static_assert(64 * 64 * 4 <= 64 * AW * 4, "exact-path staging of one channel half fits the workspace");
 
 // ---- TMEM columns (512 allocated) ----
-constexpr uint32_t TM_AP = 0;     // 2 x 64 cols, M=128: rows 0-63 A, rows 64-127 P
-constexpr uint32_t TM_W = 128;    // 128 cols, M=64: W'
-constexpr uint32_t TM_C = 256;    // 2 x 32 cols, M=128: rows 0-63 U then Delta, rows 64-127 Rq S' then O
-constexpr uint32_t TM_Z = 320;    // 32 cols, M=128: Ck^T Delta
+constexpr uint32_t TM_S = 0;      // S^T fp32 master: lane = value column, column = key channel
+constexpr uint32_t TM_SB = 128;   // S''^T bf16, two channels per column (the A operand)
+constexpr uint32_t TM_OA = 192;   // O^T of odd chunks
+constexpr uint32_t TM_D = 256;    // U^T, then Delta^T
+constexpr uint32_t TM_OB = 320;   // O^T of even chunks
+constexpr uint32_t TM_G = 384;    // Gram [A;P] or [P;A] (M=128, N=64)
+constexpr uint32_t TM_W = 448;    // -W'^T (M=128 channels, N=64 rows)
 constexpr uint32_t TM_COLS = 512;
+
+constexpr uint32_t IDESC_CRIT = idesc_bf16(128, 128, 0, 0);    // S''^T (TMEM) x stage tile
+constexpr uint32_t IDESC_Z = idesc_bf16(128, 128, 0, 1);       // Delta^T x Ck (MN-major)
+constexpr uint32_t IDESC_PD = idesc_bf16(128, 64, 0, 0);       // Delta^T x P
+constexpr uint32_t IDESC_GRAM = idesc_bf16(128, 64, 0, 0);     // stage tile x Ck
+constexpr uint32_t IDESC_W = idesc_bf16(128, 64, 1, 0, 1);     // -Rk^T (MN-major) x (T beta)^T
+constexpr uint32_t IDESC_U = idesc_bf16(128, 64, 1, 0);        // V^T (MN-major) x (T beta)
 
 // ---- mbarriers ----
 enum : int {
-  B_FULL = 0,       // [3] TMA of k, q, v landed
-  B_QRFREE = 3,     // [3] slot's k/q tiles no longer needed
-  B_TILES = 6,      // [2] Rk, Rq, Ck, scalars and exact flag written
-  B_GRAM = 8,       // [2] Gram MMA done
-  B_TB = 10,        // [2] P and T*beta tiles written
-  B_WDONE = 12,     // [2] W' and U MMAs done
-  B_READY = 14,     // [3] W' tile written
-  B_CKFREE = 17,    // [2] Ck/P slot no longer needed
-  B_DCFREE = 19,    // [2] Delta/O accumulator read
-  B_ADONE = 21,     // [-W' ; Rq] S' MMA done
-  B_DREADY = 22,    // Delta tile written
-  B_BDONE = 23,     // Ck^T Delta MMA done
-  B_ODONE = 24,     // P Delta MMA done (O complete)
-  B_SREADY = 25,    // S' tile written
-  B_PBIDLE = 26,    // prep B finished a chunk (workspace free)
-  B_FIN_C = 27,     // drains
-  B_FIN_P = 28,
-  NUM_BARS = 29
+  B_FULL = 0,       // [3] TMA of k, q landed in a stage slot
+  B_KQFREE = 3,     // [3] stage slot no longer needed (state product done)
+  B_VFULL = 6,      // TMA of v landed
+  B_TILES = 7,      // [2] Rk, Rq, Ck, scalars and exact flag written
+  B_GRAM = 9,       // Gram MMA done
+  B_TB = 10,        // P and T*beta tiles written
+  B_WDONE = 11,     // W' MMA done
+  B_UDONE = 12,     // U MMA done (v and T*beta free)
+  B_READY = 13,     // [2] -W' tile written
+  B_CRIT = 15,      // [O | Delta] product done
+  B_ZDONE = 16,     // state update product done
+  B_PD = 17,        // P Delta product done (output complete)
+  B_CKFREE = 18,    // [2] Ck/P slot no longer needed
+  B_WFREE = 20,     // prep B done with a chunk (-W' read out, workspace free)
+  B_FIN_C = 21,     // drains
+  B_FIN_P = 22,
+  NUM_BARS = 23
 };
 static_assert(NUM_BARS <= NBARS, "barrier slots");
 
@@ -142,7 +155,7 @@ struct Ctx {
   uint64_t* bars;
   volatile int* abort_flag;
   uint32_t tmem;
-  int n, h, j0, n_chunks;
+  int n, h, n_chunks;
   int64_t bos, eos;
   size_t rs;   // elements between consecutive tokens of q/k/v/o/log_alpha
 };
@@ -172,8 +185,7 @@ __device__ __forceinline__ bool wait_b(const Ctx& x, int b, uint32_t parity) {
   return wait_b_slow(x, bar, parity);
 }
 
-// Global loads issued exactly where written (volatile): used to prefetch the next
-// chunk's log-decay a whole chunk ahead of its use.
+// Global loads issued exactly where written (volatile), ahead of the barrier waits.
 __device__ __forceinline__ float4 ldg_nc_v4(const float* p) {
   float4 v;
   asm volatile("ld.global.nc.v4.f32 {%0,%1,%2,%3}, [%4];"
@@ -190,15 +202,6 @@ __device__ __forceinline__ float ldg_nc_f32(const float* p) {
 __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-// 1/x for normal positive x on the FMA pipe: integer-subtraction seed (relative
-// error < 1/8 over a binade) refined by two Newton-Raphson steps y <- y (2 - x y),
-// which square the relative error each time (< 2.5e-4 after two steps).
-__device__ __forceinline__ float rcp_nr(float x) {
-  float y = __int_as_float(0x7EF311C3 - __float_as_int(x));
-  y = y * fmaf(-x, y, 2.f);
-  y = y * fmaf(-x, y, 2.f);
   return y;
 }
 __device__ __forceinline__ float rcpf(float x) {
@@ -226,152 +229,122 @@ __device__ __forceinline__ uint64_t kdesc128(uint32_t addr) {
 }
 
 // ============================================================================
-// TMA producer (one thread)
+// TMA and MMA issue (each by the first thread of the role that consumes the result)
 // ============================================================================
-__device__ void load_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
-                          const CUtensorMap* map_v, const CUtensorMap* map_la) {
+__device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* map_k,
+                                         const CUtensorMap* map_q, int c) {
   const int xk = x.h * D;
-  for (int c = 0; c < 3 && c < x.n_chunks; ++c)
-    tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)c * CHUNK));
-  int issued = 0;
-  for (int c = 0; c < x.n_chunks; ++c) {
-    const int s3 = c % 3;
-    if (c >= 3 && !wait_b(x, B_QRFREE + s3, ((c - 3) / 3) & 1)) break;
-    const int y = (int)(x.bos + (int64_t)c * CHUNK);
-    uint8_t* qr = x.sm + OFF_QR + s3 * QR_BYTES;
-    uint64_t* full = &x.bars[B_FULL + s3];
-    mbar_arrive_expect_tx(full, 4 * 8192 + V_BYTES);
-    tma_load_2d(qr, map_k, xk, y, full);
-    tma_load_2d(qr + 16384, map_k, xk + 64, y, full);
-    tma_load_2d(qr + 8192, map_q, xk, y, full);
-    tma_load_2d(qr + 16384 + 8192, map_q, xk + 64, y, full);
-    tma_load_2d(x.sm + OFF_V + s3 * V_BYTES, map_v, xk + x.j0, y, full);
-    if (c + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, y + 3 * CHUNK);
-    issued = c + 1;
-  }
-  // never leave with copies in flight: wait (bounded) for the last load of each slot
-  for (int c = issued - 3 < 0 ? 0 : issued - 3; c < issued; ++c) {
-    uint64_t* full = &x.bars[B_FULL + c % 3];
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(full, (c / 3) & 1))
-      if (globaltimer_ns() - t0 > 100000000ull) break;
-  }
+  const int y = (int)(x.bos + (int64_t)c * CHUNK);
+  uint8_t* st = x.sm + OFF_KQ + (c % 3) * KQ_BYTES;
+  const uint32_t koff = (c & 1) ? 8192u : 0u, qoff = 8192u - koff;
+  uint64_t* full = &x.bars[B_FULL + c % 3];
+  mbar_arrive_expect_tx(full, 4 * 8192);
+  tma_load_2d(st + koff, map_k, xk, y, full);
+  tma_load_2d(st + 16384 + koff, map_k, xk + 64, y, full);
+  tma_load_2d(st + qoff, map_q, xk, y, full);
+  tma_load_2d(st + 16384 + qoff, map_q, xk + 64, y, full);
 }
-
-// ============================================================================
-// MMA issuers (one thread each)
-// ============================================================================
-__device__ void drain(const Ctx& x, int bar) {
-  umma_commit(&x.bars[bar]);
+__device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* map_v, int c) {
+  const int xk = x.h * D;
+  const int y = (int)(x.bos + (int64_t)c * CHUNK);
+  uint64_t* full = &x.bars[B_VFULL];
+  mbar_arrive_expect_tx(full, 2 * 8192);
+  tma_load_2d(x.sm + OFF_V, map_v, xk, y, full);
+  tma_load_2d(x.sm + OFF_V + 8192, map_v, xk + 64, y, full);
+}
+// On the way out: wait (bounded, ignoring the abort flag) for a copy still in flight.
+__device__ void settle(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(&x.bars[bar], 0))
+  while (!mbar_try_wait(bar, parity))
     if (globaltimer_ns() - t0 > 100000000ull) break;
 }
-
-// Sequential state pass: per chunk one stacked MMA gives Delta and Rq S', then
-// Ck^T Delta (the next state) and only then P Delta (the output).
-__device__ void mma_state_role(const Ctx& x) {
-  const uint32_t sbase = smem_u32(x.sm);
-  const uint32_t sp = sbase + OFF_SP, dl = sbase + OFF_DL;
-  for (int c = 0; c < x.n_chunks; ++c) {
-    if (!wait_b(x, B_READY + c % 3, (c / 3) & 1) || !wait_b(x, B_SREADY, c & 1)) break;
-    tc_fence_after();
-    const uint32_t qr = sbase + OFF_QR + (c % 3) * QR_BYTES;
-    const uint32_t d_c = x.tmem + TM_C + (c & 1) * 32;
-    // [U ; 0] += [-W' ; Rq] S'   (M=128, N=32, K=128)
-    for (int kk = 0; kk < 8; ++kk)
-      umma_bf16(d_c, kdesc128(qr + (kk >> 2) * 16384 + (kk & 3) * 32),
-                make_sdesc(sp + kk * 1024, 4096, 512, SWZ_64B), idesc_bf16(128, 32, 0, 1), 1u);
-    umma_commit(&x.bars[B_ADONE]);
-    if (!wait_b(x, B_DREADY, c & 1)) break;
-    tc_fence_after();
-    const uint32_t ck = sbase + OFF_CKP + (c & 1) * CKP_BYTES;
-    // Z = Ck^T Delta (M=128 channels, N=32, K=64); Ck read as an MN-major A operand
-    for (int kk = 0; kk < 4; ++kk)
-      umma_bf16(x.tmem + TM_Z, make_sdesc(ck + kk * 2048, 8192, 1024, SWZ_128B),
-                make_sdesc(dl + kk * 1024, 4096, 512, SWZ_64B), idesc_bf16(128, 32, 1, 1),
-                kk > 0 ? 1u : 0u);
-    umma_commit(&x.bars[B_BDONE]);
-    // O += P Delta: a 128-row A operand whose rows 64-127 are P (rows 0-63 are Ck's
-    // second kblock, which only touches the already-consumed Delta rows)
-    for (int kk = 0; kk < 4; ++kk)
-      umma_bf16(d_c, kdesc128(ck + 8192 + kk * 32), make_sdesc(dl + kk * 1024, 4096, 512, SWZ_64B),
-                idesc_bf16(128, 32, 0, 1), 1u);
-    umma_commit(&x.bars[B_ODONE]);
-    umma_commit(&x.bars[B_CKFREE + (c & 1)]);
-  }
-  drain(x, B_FIN_C);
+// On the way out: wait (bounded) until this thread's tensor-core work is done.
+__device__ void drain(const Ctx& x, int bar) {
+  umma_commit(&x.bars[bar]);
+  settle(&x.bars[bar], 0);
 }
 
-// Prep products in chunk order: Gram(0), W(0), Gram(1), W(1), ... The Gram of
-// chunk c+1 is queued right behind W(c), so it is done before prep B turns to
-// chunk c+1. (Queuing Gram(c+1) before W(c) could deadlock: on the exact path the
-// tiles of chunk c+1 wait for prep B to finish chunk c, which needs W(c).)
-__device__ void mma_prep_role(const Ctx& x) {
+// [O | Delta]^T (or [Delta | O]^T) += S''^T [stage tile]^T   (M=128, N=128, K=128);
+// the state operand comes from TMEM
+__device__ __forceinline__ void issue_crit(const Ctx& x, int c) {
+  tc_fence_after();
+  const uint32_t kq = smem_u32(x.sm) + OFF_KQ + (c % 3) * KQ_BYTES;
+  const uint32_t d = x.tmem + ((c & 1) ? TM_OA : TM_D);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    umma_bf16_tmem_a(d, x.tmem + TM_SB + kk * 8, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
+                     IDESC_CRIT, 1u);
+  umma_commit(&x.bars[B_CRIT]);
+  umma_commit(&x.bars[B_KQFREE + c % 3]);
+}
+// S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T
+__device__ __forceinline__ void issue_update(const Ctx& x, int c) {
+  tc_fence_after();
   const uint32_t sbase = smem_u32(x.sm);
-  const int n = x.n_chunks;
-  auto gram = [&](int g) -> bool {
-    if (!wait_b(x, B_TILES + (g & 1), (g >> 1) & 1)) return false;
-    tc_fence_after();
-    const uint32_t qr = sbase + OFF_QR + (g % 3) * QR_BYTES;
-    const uint32_t ck = sbase + OFF_CKP + (g & 1) * CKP_BYTES;
-    // [A ; P] = [Rk ; Rq] Ck^T   (M=128, N=64, K=128)
-    for (int kk = 0; kk < 8; ++kk)
-      umma_bf16(x.tmem + TM_AP + (g & 1) * 64, kdesc128(qr + (kk >> 2) * 16384 + (kk & 3) * 32),
-                kdesc128(ck + (kk >> 2) * 8192 + (kk & 3) * 32), idesc_bf16(128, 64, 0, 0),
-                kk > 0 ? 1u : 0u);
-    umma_commit(&x.bars[B_GRAM + (g & 1)]);
-    return true;
-  };
-  for (int w = 0; w < n; ++w) {
-    if (!gram(w)) break;
-    if (!wait_b(x, B_TB + (w & 1), (w >> 1) & 1)) break;
-    if (w >= 2 && !wait_b(x, B_DCFREE + (w & 1), ((w - 2) >> 1) & 1)) break;
-    tc_fence_after();
-    const uint32_t qr = sbase + OFF_QR + (w % 3) * QR_BYTES;
-    const uint32_t tb = sbase + OFF_TB;
-    const uint32_t vv = sbase + OFF_V + (w % 3) * V_BYTES;
-    // -W' = -(T beta) Rk   (M=64, N=128, K=64; negate A); Rk read as an MN-major B operand
-    for (int kk = 0; kk < 4; ++kk)
-      umma_bf16(x.tmem + TM_W, kdesc128(tb + kk * 32),
-                make_sdesc(qr + kk * 2048, 16384, 1024, SWZ_128B), idesc_bf16(64, 128, 0, 1, 1),
-                kk > 0 ? 1u : 0u);
-    // [U ; 0] = [T beta ; 0] V   (M=128, N=32, K=64): initialises the Delta/O accumulator
-    for (int kk = 0; kk < 4; ++kk)
-      umma_bf16(x.tmem + TM_C + (w & 1) * 32, kdesc128(tb + kk * 32),
-                make_sdesc(vv + kk * 1024, 4096, 512, SWZ_64B), idesc_bf16(128, 32, 0, 1),
-                kk > 0 ? 1u : 0u);
-    umma_commit(&x.bars[B_WDONE + (w & 1)]);
-  }
-  drain(x, B_FIN_P);
+  const uint32_t dt = sbase + OFF_DT;
+  const uint32_t ck = sbase + OFF_CKP + (c & 1) * CKP_BYTES;
+  // (M=128, N=128, K=64); Ck read as an MN-major B operand
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    umma_bf16(x.tmem + TM_S, kdesc128(dt + kk * 32), make_sdesc(ck + kk * 2048, 8192, 1024, SWZ_128B),
+              IDESC_Z, 1u);
+  umma_commit(&x.bars[B_ZDONE]);
+  // (M=128, N=64, K=64)
+  const uint32_t o = x.tmem + ((c & 1) ? TM_OA : TM_OB);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    umma_bf16(o, kdesc128(dt + kk * 32), kdesc128(ck + 16384 + kk * 32), IDESC_PD, 1u);
+  umma_commit(&x.bars[B_PD]);
+  umma_commit(&x.bars[B_CKFREE + (c & 1)]);
+}
+// U^T = V^T (T beta)^T   (M=128 value columns, N=64, K=64); v read as MN-major A
+__device__ __forceinline__ void issue_u(const Ctx& x) {
+  tc_fence_after();
+  const uint32_t sbase = smem_u32(x.sm);
+  const uint32_t tb = sbase + OFF_TB, vv = sbase + OFF_V;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    umma_bf16(x.tmem + TM_D, make_sdesc(vv + kk * 2048, 8192, 1024, SWZ_128B), kdesc128(tb + kk * 32),
+              IDESC_U, kk > 0 ? 1u : 0u);
+  umma_commit(&x.bars[B_UDONE]);
+}
+// -W'^T = -Rk^T (T beta)^T   (M=128 channels, N=64, K=64); Rk (the k half of the
+// stage tile) read as an MN-major A operand
+__device__ __forceinline__ void issue_w(const Ctx& x, int c) {
+  tc_fence_after();
+  const uint32_t sbase = smem_u32(x.sm);
+  const uint32_t kq = sbase + OFF_KQ + (c % 3) * KQ_BYTES + ((c & 1) ? 8192u : 0u);
+  const uint32_t tb = sbase + OFF_TB;
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+    umma_bf16(x.tmem + TM_W, make_sdesc(kq + kk * 2048, 16384, 1024, SWZ_128B), kdesc128(tb + kk * 32),
+              IDESC_W, kk > 0 ? 1u : 0u);
+  umma_commit(&x.bars[B_WDONE]);
 }
 
-// Exact path of prep A for a chunk whose decay range is too wide for the factored
-// Gram (kept out of line: it is rare and large). Pairwise factors are evaluated
-// one by one; A goes to prep B's workspace, P to its tile, and the operand tiles are
-// built with the reference before the chunk (all factors <= 1).
-__device__ __noinline__ bool prep_a_exact(const Ctx& x, int c, int L, uint8_t* qr, uint8_t* ck,
-                                          const float* betas, const float (&g2)[8][4],
-                                          const float (&gc)[4]) {
+// ============================================================================
+// prep A (warps 0-7): decay factors and the three bf16 tiles of a chunk
+// ============================================================================
+
+// Exact path for a chunk whose decay range is too wide for the factored Gram (kept
+// out of line: it is rare and large). Pairwise factors are evaluated one by one,
+// one channel half at a time with G staged in prep B's workspace; A goes to that
+// workspace, P to its tile, and Rk / Rq are built about the point before the chunk.
+__device__ __noinline__ bool prep_a_exact(const Ctx& x, int c, int L, uint8_t* kq, uint32_t koff,
+                                          uint32_t qoff, uint8_t* ck, const float* betas,
+                                          const float (&g2)[8][4], const float (&gc)[4]) {
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
   const int kb = lane >> 4;
   const uint32_t cbyte = (lane & 15) * 8;
   const int c0 = 4 * lane;
-  const int s2 = c & 1;
   float* aw = reinterpret_cast<float*>(x.sm + OFF_AW);
-  bool ok = true;
-  // ---- exact path. Needs prep B's workspace (idle after chunk c-1) and this Ck/P slot.
-  ok = (c < 1) || wait_b(x, B_PBIDLE, (c - 1) & 1);
-  ok = ok && ((c < 2) || wait_b(x, B_CKFREE + s2, ((c - 2) >> 1) & 1));
+  // prep B must be done with chunk c-1 (its workspace) and this Ck/P slot free
+  bool ok = (c < 1) || wait_b(x, B_WFREE, (c - 1) & 1);
+  ok = ok && ((c < 2) || wait_b(x, B_CKFREE + (c & 1), ((c - 2) >> 1) & 1));
   if (named_bar_or(BAR_PA, PA_THREADS, !ok)) return false;
-  float* gsm = reinterpret_cast<float*>(x.sm + OFF_TB);   // G (log2 units), [64][128] fp32
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    *reinterpret_cast<float4*>(&gsm[(8 * w + j) * 128 + c0]) =
-        make_float4(g2[j][0], g2[j][1], g2[j][2], g2[j][3]);
-  named_bar_sync(BAR_PA, PA_THREADS);
-  // warp w takes lower-triangle pairs p = w, w+8, ... (row-major r(r+1)/2 + i)
+  // warp w takes lower-triangle pairs p = w, w+8, ... (row-major r(r+1)/2 + i); the
+  // lane that finishes a pair's reduction keeps it (the same lane in both halves)
   float pval[9], aval[9];
   int pidx[9];
 #pragma unroll
@@ -379,46 +352,57 @@ __device__ __noinline__ bool prep_a_exact(const Ctx& x, int c, int L, uint8_t* q
     pval[bt] = 0.f;
     aval[bt] = 0.f;
     pidx[bt] = -1;
-#pragma unroll 1
-    for (int qq = 0; qq < 32; ++qq) {
-      const int pp = w + 8 * (bt * 32 + qq);
-      if (pp >= 2080) break;
-      int r = (int)((sqrtf(8.f * pp + 1.f) - 1.f) * 0.5f);
-      while ((r + 1) * (r + 2) / 2 <= pp) ++r;
-      while (r * (r + 1) / 2 > pp) --r;
-      const int i = pp - r * (r + 1) / 2;
-      float sa = 0.f, sp = 0.f;
-      if (r < L && i < L) {
-        const uint2 kr = *reinterpret_cast<const uint2*>(qr + kb * 16384 + swz128(r * 128 + cbyte));
-        const uint2 ki = *reinterpret_cast<const uint2*>(qr + kb * 16384 + swz128(i * 128 + cbyte));
-        const uint2 qv = *reinterpret_cast<const uint2*>(qr + kb * 16384 + swz128((r + 64) * 128 + cbyte));
-        const float4 gr = *reinterpret_cast<const float4*>(&gsm[r * 128 + c0]);
-        const float4 gi = *reinterpret_cast<const float4*>(&gsm[i * 128 + c0]);
-        const float ee[4] = {ex2f(gr.x - gi.x), ex2f(gr.y - gi.y), ex2f(gr.z - gi.z), ex2f(gr.w - gi.w)};
-        const float krf[4] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y)};
-        const float kif[4] = {bf_lo(ki.x), bf_hi(ki.x), bf_lo(ki.y), bf_hi(ki.y)};
-        const float qf[4] = {bf_lo(qv.x), bf_hi(qv.x), bf_lo(qv.y), bf_hi(qv.y)};
+  }
+  float* gsm = aw;   // G (log2 units) of one channel half: [64 rows][64] fp32
+  for (int hf = 0; hf < 2; ++hf) {
+    if (kb == hf) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float ke = kif[k] * ee[k];
-          sa = fmaf(krf[k], ke, sa);
-          sp = fmaf(qf[k], ke, sp);
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(&gsm[(8 * w + j) * 64 + (c0 - 64 * hf)]) =
+            make_float4(g2[j][0], g2[j][1], g2[j][2], g2[j][3]);
+    }
+    named_bar_sync(BAR_PA, PA_THREADS);
+    const int ch = 2 * lane;                  // channel pair within the half
+    const uint32_t cb = (uint32_t)ch * 2u;    // its byte offset in the kblock row
+    const uint8_t* kt = kq + koff + hf * 16384;
+    const uint8_t* qt = kq + qoff + hf * 16384;
+#pragma unroll
+    for (int bt = 0; bt < 9; ++bt) {
+#pragma unroll 1
+      for (int qq = 0; qq < 32; ++qq) {
+        const int pp = w + 8 * (bt * 32 + qq);
+        if (pp >= 2080) break;
+        int r = (int)((sqrtf(8.f * pp + 1.f) - 1.f) * 0.5f);
+        while ((r + 1) * (r + 2) / 2 <= pp) ++r;
+        while (r * (r + 1) / 2 > pp) --r;
+        const int i = pp - r * (r + 1) / 2;
+        float sa = 0.f, sp = 0.f;
+        if (r < L && i < L) {
+          const uint32_t kr = *reinterpret_cast<const uint32_t*>(kt + swz128(r * 128 + cb));
+          const uint32_t ki = *reinterpret_cast<const uint32_t*>(kt + swz128(i * 128 + cb));
+          const uint32_t qv = *reinterpret_cast<const uint32_t*>(qt + swz128(r * 128 + cb));
+          const float2 gr = *reinterpret_cast<const float2*>(&gsm[r * 64 + ch]);
+          const float2 gi = *reinterpret_cast<const float2*>(&gsm[i * 64 + ch]);
+          const float ke0 = bf_lo(ki) * ex2f(gr.x - gi.x);
+          const float ke1 = bf_hi(ki) * ex2f(gr.y - gi.y);
+          sa = fmaf(bf_lo(kr), ke0, bf_hi(kr) * ke1);
+          sp = fmaf(bf_lo(qv), ke0, bf_hi(qv) * ke1);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          sa += __shfl_xor_sync(0xffffffffu, sa, off);
+          sp += __shfl_xor_sync(0xffffffffu, sp, off);
+        }
+        if (lane == qq) {
+          pval[bt] += sp;
+          aval[bt] += sa;
+          pidx[bt] = r * 64 + i;
         }
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        sa += __shfl_xor_sync(0xffffffffu, sa, off);
-        sp += __shfl_xor_sync(0xffffffffu, sp, off);
-      }
-      if (lane == qq) {
-        pval[bt] = sp;
-        aval[bt] = sa;
-        pidx[bt] = r * 64 + i;
-      }
     }
+    named_bar_sync(BAR_PA, PA_THREADS);   // the staging area is rewritten next
   }
-  named_bar_sync(BAR_PA, PA_THREADS);
-  // A (beta-scaled, strictly lower) into prep B's workspace; P tile zeroed then filled
+  // P tile cleared, then A (beta-scaled, strictly lower) and P filled in
   uint8_t* pt = ck + 16384;
   for (int idx = tid; idx < 512; idx += PA_THREADS)
     *reinterpret_cast<uint4*>(pt + idx * 16) = make_uint4(0u, 0u, 0u, 0u);
@@ -430,16 +414,13 @@ __device__ __noinline__ bool prep_a_exact(const Ctx& x, int c, int L, uint8_t* q
       *reinterpret_cast<__nv_bfloat16*>(pt + swz128(r * 128 + i * 2)) = __float2bfloat16_rn(pval[bt]);
       if (i < r) aw[r * AW + i] = betas[r] * aval[bt];
     }
-  // the staging area covered the zero rows of prep B's [T*beta ; 0] operand: restore them
-  for (int idx = tid; idx < 512; idx += PA_THREADS)
-    *reinterpret_cast<uint4*>(x.sm + OFF_TB + 8192 + idx * 16) = make_uint4(0u, 0u, 0u, 0u);
-  // tiles with the reference before the chunk: Rk = K e^G, Rq = Q e^G, Ck = K e^{G_C - G}
+  // tiles about the point before the chunk: Rk = K e^G, Rq = Q e^G; Ck = K e^{G_C - G}
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int r = 8 * w + j;
     const bool valid = r < L;
-    uint2* kp = reinterpret_cast<uint2*>(qr + kb * 16384 + swz128(r * 128 + cbyte));
-    uint2* qp = reinterpret_cast<uint2*>(qr + kb * 16384 + swz128((r + 64) * 128 + cbyte));
+    uint2* kp = reinterpret_cast<uint2*>(kq + koff + kb * 16384 + swz128(r * 128 + cbyte));
+    uint2* qp = reinterpret_cast<uint2*>(kq + qoff + kb * 16384 + swz128(r * 128 + cbyte));
     uint2* cp = reinterpret_cast<uint2*>(ck + kb * 8192 + swz128(r * 128 + cbyte));
     const uint2 kr = valid ? *kp : make_uint2(0u, 0u);
     const uint2 qv = valid ? *qp : make_uint2(0u, 0u);
@@ -455,13 +436,11 @@ __device__ __noinline__ bool prep_a_exact(const Ctx& x, int c, int L, uint8_t* q
     *qp = make_uint2(pack_bf16(qf[0] * e[0], qf[1] * e[1]), pack_bf16(qf[2] * e[2], qf[3] * e[3]));
     *cp = make_uint2(pack_bf16(krf[0] * f[0], krf[1] * f[1]), pack_bf16(krf[2] * f[2], krf[3] * f[3]));
   }
-  return ok;
+  return true;
 }
 
-// ============================================================================
-// prep A (warps 0-7): decay factors and the three bf16 tiles of a chunk
-// ============================================================================
-__device__ void prep_a_role(const Ctx& x, const Args& p) {
+__device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_k,
+                            const CUtensorMap* map_q, const CUtensorMap* map_la) {
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
   const int kb = lane >> 4;                // kblock of this thread's 4 channels
@@ -470,41 +449,40 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
   float* wsum = reinterpret_cast<float*>(x.sm + OFF_WSUM);
   float* grow = reinterpret_cast<float*>(x.sm + OFF_GROW);
   int* xflag = reinterpret_cast<int*>(x.sm + OFF_XFLAG);
+  const int xk = x.h * D;
+  // (thread 0) k/q loads run two chunks ahead of this role; the log-decay is
+  // prefetched into L2 three chunks ahead
+  int kq_issued = 0, kq_landed = 0;
+  if (tid == 0) {
+    for (int c = 0; c < 3 && c < x.n_chunks; ++c)
+      tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)c * CHUNK));
+    for (; kq_issued < 2 && kq_issued < x.n_chunks; ++kq_issued) issue_kq(x, map_k, map_q, kq_issued);
+  }
 
-  float lam_next[8][4];
-  float beta_next = 0.f;
-  auto load_next = [&](int c) {
+  for (int c = 0; c < x.n_chunks; ++c) {
+    const int s3 = c % 3;
     const int64_t t0 = x.bos + (int64_t)c * CHUNK;
+    const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
+    uint8_t* kq = x.sm + OFF_KQ + s3 * KQ_BYTES;
+    uint8_t* ck = x.sm + OFF_CKP + (c & 1) * CKP_BYTES;
+    const uint32_t koff = (c & 1) ? 8192u : 0u, qoff = 8192u - koff;
+    float* betas = reinterpret_cast<float*>(x.sm + OFF_BETA) + s3 * 64;
+    float* scal = reinterpret_cast<float*>(x.sm + OFF_SCAL) + s3 * 256;
+
+    // log-decay rows 8w..8w+7 of this chunk, channels c0..c0+3 (L2-prefetched by the
+    // TMA thread three chunks ahead); zero past the end of the sequence
+    float g2[8][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int64_t t = t0 + 8 * w + j;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c < x.n_chunks && t < x.eos)
-        v = ldg_nc_v4(p.log_alpha + (size_t)t * x.rs + x.h * D + c0);
-      lam_next[j][0] = v.x; lam_next[j][1] = v.y; lam_next[j][2] = v.z; lam_next[j][3] = v.w;
+      if (t < x.eos) v = ldg_nc_v4(p.log_alpha + (size_t)t * x.rs + x.h * D + c0);
+      g2[j][0] = v.x; g2[j][1] = v.y; g2[j][2] = v.z; g2[j][3] = v.w;
     }
-    beta_next = 0.f;
-    if (tid < 64 && c < x.n_chunks && t0 + tid < x.eos)
-      beta_next = ldg_nc_f32(p.beta + (size_t)(t0 + tid) * p.n_heads + x.h);
-  };
-  load_next(0);
-
-  for (int c = 0; c < x.n_chunks; ++c) {
-    const int s3 = c % 3, s2 = c & 1;
-    const int64_t t0 = x.bos + (int64_t)c * CHUNK;
-    const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
-    uint8_t* qr = x.sm + OFF_QR + s3 * QR_BYTES;
-    uint8_t* ck = x.sm + OFF_CKP + s2 * CKP_BYTES;
-    float* betas = reinterpret_cast<float*>(x.sm + OFF_BETA) + s3 * 64;
-    float* scal = reinterpret_cast<float*>(x.sm + OFF_SCAL) + s3 * 384;
-
-    float g2[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) g2[j][k] = lam_next[j][k];
-    if (tid < 64) betas[tid] = beta_next;
-    load_next(c + 1);   // next chunk's log-decay and beta, in flight during this one
+    // (the reader of this beta slot, prep B three chunks back, finished before this
+    // role got the Ck slot of chunk c-1)
+    if (tid < 64)
+      betas[tid] = (t0 + tid < x.eos) ? ldg_nc_f32(p.beta + (size_t)(t0 + tid) * p.n_heads + x.h) : 0.f;
 
     // ---- inclusive cumsum over rows, in log2 units
     {
@@ -530,71 +508,78 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) g2[j][k] += pre[k];
       if (w == 0) *reinterpret_cast<float4*>(&grow[c0]) = make_float4(g2[0][0], g2[0][1], g2[0][2], g2[0][3]);
-      if (w == 3) *reinterpret_cast<float4*>(&grow[128 + c0]) = make_float4(g2[7][0], g2[7][1], g2[7][2], g2[7][3]);
-      if (w == 7) *reinterpret_cast<float4*>(&grow[256 + c0]) = make_float4(g2[7][0], g2[7][1], g2[7][2], g2[7][3]);
+      if (w == 7) *reinterpret_cast<float4*>(&grow[128 + c0]) = make_float4(g2[7][0], g2[7][1], g2[7][2], g2[7][3]);
     }
     bool ok = wait_b(x, B_FULL + s3, (c / 3) & 1);
+    if (ok) kq_landed = c + 1;
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
 
     // ---- range guard: max over channels of G_0 - G_63
     bool bad = false;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) bad |= (grow[c0 + k] - grow[256 + c0 + k]) > GUARD_LOG2;
+    for (int k = 0; k < 4; ++k) bad |= (grow[c0 + k] - grow[128 + c0 + k]) > GUARD_LOG2;
     const bool exact = named_bar_or(BAR_PA, PA_THREADS, bad);
 
-    float gm[4], gc[4];
+    float gc[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      gm[k] = exact ? 0.f : grow[128 + c0 + k];
-      gc[k] = grow[256 + c0 + k];
-    }
+    for (int k = 0; k < 4; ++k) gc[k] = grow[128 + c0 + k];
 
     if (!exact) {
-      // ---- factored tiles: Rk = K E, Rq = Q E in place; Ck = K F once the slot is free
-      uint32_t kf[8][2];
+      ok = (c < 2) || wait_b(x, B_CKFREE + (c & 1), ((c - 2) >> 1) & 1);
+      // ---- factored tiles: Rk = K E, Rq = Q E in place, Ck = K F
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int r = 8 * w + j;
         const bool valid = r < L;
-        uint2* kp = reinterpret_cast<uint2*>(qr + kb * 16384 + swz128(r * 128 + cbyte));
-        uint2* qp = reinterpret_cast<uint2*>(qr + kb * 16384 + swz128((r + 64) * 128 + cbyte));
+        uint2* kp = reinterpret_cast<uint2*>(kq + koff + kb * 16384 + swz128(r * 128 + cbyte));
+        uint2* qp = reinterpret_cast<uint2*>(kq + qoff + kb * 16384 + swz128(r * 128 + cbyte));
         const uint2 kr = valid ? *kp : make_uint2(0u, 0u);
         const uint2 qv = valid ? *qp : make_uint2(0u, 0u);
         float e[4], f[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          e[k] = ex2f(g2[j][k] - gm[k]);
+          e[k] = ex2f(g2[j][k] - gc[k]);
           f[k] = rcpf(e[k]);
         }
         const uint32_t e01 = pack_bf16(e[0], e[1]), e23 = pack_bf16(e[2], e[3]);
         *kp = make_uint2(mul_bf16x2(kr.x, e01), mul_bf16x2(kr.y, e23));
         *qp = make_uint2(mul_bf16x2(qv.x, e01), mul_bf16x2(qv.y, e23));
-        kf[j][0] = mul_bf16x2(kr.x, pack_bf16(f[0], f[1]));
-        kf[j][1] = mul_bf16x2(kr.y, pack_bf16(f[2], f[3]));
+        if (ok)
+          *reinterpret_cast<uint2*>(ck + kb * 8192 + swz128(r * 128 + cbyte)) =
+              make_uint2(mul_bf16x2(kr.x, pack_bf16(f[0], f[1])),
+                         mul_bf16x2(kr.y, pack_bf16(f[2], f[3])));
       }
-      ok = (c < 2) || wait_b(x, B_CKFREE + s2, ((c - 2) >> 1) & 1);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        *reinterpret_cast<uint2*>(ck + kb * 8192 + swz128((8 * w + j) * 128 + cbyte)) =
-            make_uint2(kf[j][0], kf[j][1]);
     } else {
-      ok = prep_a_exact(x, c, L, qr, ck, betas, g2, gc);
+      ok = prep_a_exact(x, c, L, kq, koff, qoff, ck, betas, g2, gc);
       if (!ok) break;
     }
     // per-channel scalars and the path flag of this chunk
     if (w == 0) {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        scal[c0 + k] = exact ? 1.f : ex2f(gm[k]);               // e^{G_m}
-        scal[128 + c0 + k] = ex2f(gc[k]);                        // e^{G_C}
-        scal[256 + c0 + k] = exact ? 1.f : ex2f(gc[k] - gm[k]);  // e^{G_C - G_m}
+        const float egc = ex2f(gc[k]);
+        scal[c0 + k] = egc;                        // decay of the state over the chunk
+        scal[128 + c0 + k] = exact ? 1.f : egc;    // scale of the state operand
       }
       if (lane == 0) xflag[s3] = exact ? 1 : 0;
     }
     fence_proxy_async_smem();
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
-    if (tid == 0) mbar_arrive(&x.bars[B_TILES + s2]);
+    if (tid == 0) {
+      mbar_arrive(&x.bars[B_TILES + (c & 1)]);
+      // k/q of chunk c+2 into the slot that chunk c-1 used (free once its state
+      // product is done), and the L2 prefetch of chunk c+3's log-decay
+      const int cn = c + 2;
+      if (cn < x.n_chunks && (cn < 3 || wait_b(x, B_KQFREE + cn % 3, ((cn - 3) / 3) & 1))) {
+        issue_kq(x, map_k, map_q, cn);
+        kq_issued = cn + 1;
+      }
+      if (c + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(c + 3) * CHUNK));
+    }
   }
+  // never leave with copies in flight
+  if (tid == 0)
+    for (int c = kq_landed; c < kq_issued; ++c) settle(&x.bars[B_FULL + c % 3], (c / 3) & 1);
 }
 
 // ============================================================================
@@ -631,17 +616,40 @@ __device__ __forceinline__ void blk_store(float* C, int ldc, const float (&acc)[
     C[(g + 8) * ldc + 8 * nh + 2 * t + 1] = scale * acc[nh][3];
   }
 }
-
-// Block (a, b), a >= b, of T = (I + A)^{-1} after the solve (fp32, 16x16).
-// Diagonal and (1,0), (2,0), (3,0), (3,1), (3,2) overwrite the matching A block;
-// (2,1) lives in the extra-block area.
-__device__ __forceinline__ const float* tblk(const uint8_t* sm, int a, int b, int& ld) {
-  if (a == 2 && b == 1) {
-    ld = 16;
-    return reinterpret_cast<const float*>(sm + OFF_XS) + 4 * 256;
+// A finished block (a, b) of T, scaled by `scale`, into the bf16 T*beta tile (column i
+// of T times beta_i), two columns per 32-bit store.
+__device__ __forceinline__ void blk_store_tb(uint8_t* tt, int a, int b, const float (&acc)[2][4],
+                                             float scale, const float* betas, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nh = 0; nh < 2; ++nh) {
+    const int i = 16 * b + 8 * nh + 2 * t;
+    const float b0 = scale * betas[i], b1 = scale * betas[i + 1];
+    *reinterpret_cast<uint32_t*>(tt + swz128((16 * a + g) * 128 + i * 2)) =
+        pack_bf16(acc[nh][0] * b0, acc[nh][1] * b1);
+    *reinterpret_cast<uint32_t*>(tt + swz128((16 * a + g + 8) * 128 + i * 2)) =
+        pack_bf16(acc[nh][2] * b0, acc[nh][3] * b1);
   }
-  ld = AW;
-  return reinterpret_cast<const float*>(sm + OFF_AW) + (16 * a) * AW + 16 * b;
+}
+
+// Gram product of chunk g (issued by prep B's first thread): [A ; P] or [P ; A] =
+// stage tile x Ck^T (M=128, N=64, K=128). For an exact-path chunk only the commit
+// goes out, so the barrier completes one phase per chunk either way.
+__device__ __forceinline__ void issue_gram(const Ctx& x, int g) {
+  const int* xflag = reinterpret_cast<const int*>(x.sm + OFF_XFLAG);
+  if (xflag[g % 3]) {
+    umma_commit(&x.bars[B_GRAM]);
+    return;
+  }
+  tc_fence_after();
+  const uint32_t sbase = smem_u32(x.sm);
+  const uint32_t kq = sbase + OFF_KQ + (g % 3) * KQ_BYTES;
+  const uint32_t ck = sbase + OFF_CKP + (g & 1) * CKP_BYTES;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    umma_bf16(x.tmem + TM_G, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
+              kdesc128(ck + (kk >> 2) * 8192 + (kk & 3) * 32), IDESC_GRAM, kk > 0 ? 1u : 0u);
+  umma_commit(&x.bars[B_GRAM]);
 }
 
 __device__ void prep_b_role(const Ctx& x) {
@@ -652,31 +660,40 @@ __device__ void prep_b_role(const Ctx& x) {
   float* scr = reinterpret_cast<float*>(x.sm + OFF_SCR) + q * 256;
   const int* xflag = reinterpret_cast<const int*>(x.sm + OFF_XFLAG);
   auto A = [&](int a, int b) { return aw + (16 * a) * AW + 16 * b; };
-  // rows 64-127 of the [T*beta ; 0] operand stay zero for the whole kernel
+  uint8_t* tt = x.sm + OFF_TB;
+  int gram_issued = 0;   // (thread 0) Gram products issued so far
+  // blocks above the diagonal of the T*beta tile stay zero for the whole kernel
   for (int i = tid; i < 512; i += PB_THREADS)
-    *reinterpret_cast<uint4*>(x.sm + OFF_TB + 8192 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
-  fence_proxy_async_smem();
+    *reinterpret_cast<uint4*>(tt + i * 16) = make_uint4(0u, 0u, 0u, 0u);
 
   for (int c = 0; c < x.n_chunks; ++c) {
-    const int s3 = c % 3, s2 = c & 1;
-    uint8_t* qr = x.sm + OFF_QR + s3 * QR_BYTES;
-    uint8_t* ck = x.sm + OFF_CKP + s2 * CKP_BYTES;
+    const int s3 = c % 3;
+    uint8_t* kq = x.sm + OFF_KQ + s3 * KQ_BYTES;
+    uint8_t* ck = x.sm + OFF_CKP + (c & 1) * CKP_BYTES;
     const float* betas = reinterpret_cast<const float*>(x.sm + OFF_BETA) + s3 * 64;
+    const uint32_t koff = (c & 1) ? 8192u : 0u;
 
-    bool ok = wait_b(x, B_TILES + s2, (c >> 1) & 1);
+    bool ok = wait_b(x, B_TILES + (c & 1), (c >> 1) & 1);
     const bool exact = ok && xflag[s3] != 0;
-    // ---- Gram readout: A rows (beta-scaled, strictly lower) -> fp32 workspace; P -> bf16 tile
+    // the Gram of this chunk, unless it went out while the previous chunk was solved
+    if (tid == 0 && ok && c >= gram_issued) {
+      issue_gram(x, c);
+      gram_issued = c + 1;
+    }
+    // ---- Gram readout: A rows (beta-scaled, strictly lower) -> fp32 workspace; P -> bf16 tile.
+    //      Lanes of the k half hold A, lanes of the q half hold P.
+    ok = ok && wait_b(x, B_GRAM, c & 1);
     if (ok && !exact) {
-      ok = wait_b(x, B_GRAM + s2, (c >> 1) & 1);
       tc_fence_after();
+      const bool a_rows = (q < 2) == ((c & 1) == 0);
+      const int r = 32 * (q & 1) + lane;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int col0 = 32 * half;
         float v[32];
-        tmem_ld32(x.tmem + TM_AP + s2 * 64 + lane_base + col0, v);
+        tmem_ld32(x.tmem + TM_G + lane_base + col0, v);
         tmem_ld_wait();
-        if (q < 2) {
-          const int r = 32 * q + lane;
+        if (a_rows) {
           const float br = betas[r];
 #pragma unroll
           for (int m = 0; m < 32; m += 4) {
@@ -688,7 +705,6 @@ __device__ void prep_b_role(const Ctx& x) {
             *reinterpret_cast<float4*>(&aw[r * AW + col0 + m]) = o4;
           }
         } else {
-          const int r = 32 * (q - 2) + lane;
           uint8_t* pt = ck + 16384;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -701,11 +717,21 @@ __device__ void prep_b_role(const Ctx& x) {
       }
       tc_fence_before();
     }
+    // the previous chunk's U product must be done reading the T*beta tile
+    ok = ok && ((c < 1) || wait_b(x, B_UDONE, (c - 1) & 1));
     if (named_bar_or(BAR_PB, PB_THREADS, !ok)) break;
+    // the Gram columns are free again: the next chunk's Gram goes out now if its
+    // tiles are already written
+    if (tid == 0 && c + 1 < x.n_chunks &&
+        mbar_test_wait(&x.bars[B_TILES + ((c + 1) & 1)], ((c + 1) >> 1) & 1)) {
+      issue_gram(x, c + 1);
+      gram_issued = c + 2;
+    }
 
     // ---- UT transform: T = (I + A)^{-1}. 16x16 diagonal blocks by forward substitution:
     //      lane j of warp a keeps column j of T_aa in registers (the A values are
-    //      independent of it, so their loads pipeline), then the block replaces A_aa.
+    //      independent of it, so their loads pipeline), then the block replaces A_aa
+    //      and its T*beta entries go to the tile.
     if (lane < 16) {
       const int j = lane;
       float* Ab = A(q, q);
@@ -722,8 +748,13 @@ __device__ void prep_b_role(const Ctx& x) {
         t[r] = (r == j ? 1.f : 0.f) - (s0 + s1);
       }
       __syncwarp(0x0000ffffu);
+      const float bj = betas[16 * q + j];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) Ab[r * AW + j] = t[r];
+      for (int r = 0; r < 16; ++r) {
+        Ab[r * AW + j] = t[r];
+        *reinterpret_cast<__nv_bfloat16*>(tt + swz128((16 * q + r) * 128 + (16 * q + j) * 2)) =
+            __float2bfloat16_rn(t[r] * bj);
+      }
     }
     named_bar_sync(BAR_PB, PB_THREADS);
     // Off-diagonal blocks by 2x2 block doubling (tf32 warp MMAs), three levels:
@@ -735,7 +766,6 @@ __device__ void prep_b_role(const Ctx& x) {
       float* X21 = xs + 256;
       float* X30 = xs + 512;
       float* X31 = xs + 768;
-      float* T21 = xs + 1024;
       float* T31p = xs + 1280;
       if (q == 0) {        // T_10
         float acc[2][4] = {};
@@ -745,6 +775,7 @@ __device__ void prep_b_role(const Ctx& x) {
         float acc2[2][4] = {};
         blk_mma(acc2, A(1, 1), AW, scr, 16, lane);
         blk_store(A(1, 0), AW, acc2, -1.f, lane);
+        blk_store_tb(tt, 1, 0, acc2, -1.f, betas, lane);
       } else if (q == 1) { // T_32
         float acc[2][4] = {};
         blk_mma(acc, A(3, 2), AW, A(2, 2), AW, lane);
@@ -753,6 +784,7 @@ __device__ void prep_b_role(const Ctx& x) {
         float acc2[2][4] = {};
         blk_mma(acc2, A(3, 3), AW, scr, 16, lane);
         blk_store(A(3, 2), AW, acc2, -1.f, lane);
+        blk_store_tb(tt, 3, 2, acc2, -1.f, betas, lane);
       } else if (q == 2) { // X21 = A_21 T_11
         float acc[2][4] = {};
         blk_mma(acc, A(2, 1), AW, A(1, 1), AW, lane);
@@ -776,7 +808,7 @@ __device__ void prep_b_role(const Ctx& x) {
       } else if (q == 2) { // T_21 = -T_22 X21
         float acc[2][4] = {};
         blk_mma(acc, A(2, 2), AW, X21, 16, lane);
-        blk_store(T21, 16, acc, -1.f, lane);
+        blk_store_tb(tt, 2, 1, acc, -1.f, betas, lane);
       } else {             // partial of T_31: T_33 X31
         float acc[2][4] = {};
         blk_mma(acc, A(3, 3), AW, X31, 16, lane);
@@ -786,12 +818,12 @@ __device__ void prep_b_role(const Ctx& x) {
       if (q == 0) {        // T_20 = -T_22 X20
         float acc[2][4] = {};
         blk_mma(acc, A(2, 2), AW, X20, 16, lane);
-        blk_store(A(2, 0), AW, acc, -1.f, lane);
+        blk_store_tb(tt, 2, 0, acc, -1.f, betas, lane);
       } else if (q == 1) { // T_30 = -(T_32 X20 + T_33 X30)
         float acc[2][4] = {};
         blk_mma(acc, A(3, 2), AW, X20, 16, lane);
         blk_mma(acc, A(3, 3), AW, X30, 16, lane);
-        blk_store(A(3, 0), AW, acc, -1.f, lane);
+        blk_store_tb(tt, 3, 0, acc, -1.f, betas, lane);
       } else if (q == 2) { // T_31 = -(T_32 X21 + T_33 X31)
         float acc[2][4] = {};
         blk_mma(acc, A(3, 2), AW, X21, 16, lane);
@@ -803,180 +835,232 @@ __device__ void prep_b_role(const Ctx& x) {
           acc[nh][2] += T31p[(g + 8) * 16 + 8 * nh + 2 * t];
           acc[nh][3] += T31p[(g + 8) * 16 + 8 * nh + 2 * t + 1];
         }
-        blk_store(A(3, 1), AW, acc, -1.f, lane);
-      }
-      named_bar_sync(BAR_PB, PB_THREADS);
-    }
-    // ---- T*beta tile (bf16, K-major [64 r][64 i], 128B swizzle): thread = (row, 32-col half)
-    {
-      const int r = tid >> 1, hh = tid & 1;
-      uint8_t* tt = x.sm + OFF_TB;
-      const int a = r >> 4, rr = r & 15;
-#pragma unroll
-      for (int bb = 0; bb < 2; ++bb) {
-        const int b = 2 * hh + bb;   // 16-column block
-        float tv[16];
-        if (b <= a) {
-          int ld;
-          const float* Tb = tblk(x.sm, a, b, ld);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int i = 16 * b + e;
-            tv[e] = (i <= r) ? Tb[rr * ld + e] * betas[i] : 0.f;
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) tv[e] = 0.f;
-        }
-        *reinterpret_cast<uint4*>(tt + swz128(r * 128 + b * 32)) = pack8(tv);
-        *reinterpret_cast<uint4*>(tt + swz128(r * 128 + b * 32 + 16)) = pack8(tv + 8);
+        blk_store_tb(tt, 3, 1, acc, -1.f, betas, lane);
       }
     }
     fence_proxy_async_smem();
     named_bar_sync(BAR_PB, PB_THREADS);
-    if (tid == 0) mbar_arrive(&x.bars[B_TB + s2]);
+    if (tid == 0) {
+      mbar_arrive(&x.bars[B_TB]);
+      issue_w(x, c);
+    }
 
-    // ---- -W' readout (M=64 layout: rows 16q..16q+15 in lanes 32q..32q+15) -> bf16 over Rk
-    ok = wait_b(x, B_WDONE + s2, (c >> 1) & 1);
+    // ---- -W' readout: lane = channel ch, columns = rows r. Lane pairs (ch, ch+1) swap
+    //      halves so that each 32-bit store holds two channels of one row: the even
+    //      lane writes the even rows, the odd lane the odd rows.
+    ok = wait_b(x, B_WDONE, c & 1);
     tc_fence_after();
+    {
+      const int ch = 32 * q + lane;
+      const bool odd = lane & 1;
+      uint8_t* wt = kq + koff + (ch >> 6) * 16384;
+      const uint32_t cb = (uint32_t)((ch & 63) & ~1) * 2u;
 #pragma unroll 1
-    for (int part = 0; part < 4; ++part) {
-      float v[32];
-      tmem_ld32(x.tmem + TM_W + lane_base + 32 * part, v);
-      tmem_ld_wait();
-      if (lane < 16) {
-        const int r = 16 * q + lane;
-        uint8_t* rowp = qr + (part >> 1) * 16384;
+      for (int half = 0; half < 2; ++half) {
+        float v[32];
+        tmem_ld32(x.tmem + TM_W + lane_base + 32 * half, v);
+        tmem_ld_wait();
+        if (ok) {
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
-          *reinterpret_cast<uint4*>(rowp + swz128(r * 128 + (part & 1) * 64 + ch * 16)) =
-              pack8(v + ch * 8);
+          for (int k = 0; k < 16; ++k) {
+            const float other = __shfl_xor_sync(0xffffffffu, odd ? v[2 * k] : v[2 * k + 1], 1);
+            const int r = 32 * half + 2 * k + (odd ? 1 : 0);
+            const uint32_t pr = odd ? pack_bf16(other, v[2 * k + 1]) : pack_bf16(v[2 * k], other);
+            *reinterpret_cast<uint32_t*>(wt + swz128(r * 128 + cb)) = pr;
+          }
+        }
       }
     }
     tc_fence_before();
     fence_proxy_async_smem();
     if (named_bar_or(BAR_PB, PB_THREADS, !ok)) break;
     if (tid == 0) {
-      mbar_arrive(&x.bars[B_READY + s3]);
-      mbar_arrive(&x.bars[B_PBIDLE]);
+      mbar_arrive(&x.bars[B_READY + (c & 1)]);
+      mbar_arrive(&x.bars[B_WFREE]);
     }
   }
+  if (tid == 0) drain(x, B_FIN_P);
 }
 
 // ============================================================================
-// state warps (12-15): the sequential pass over chunks
+// state warps (12-19): the sequential pass over chunks. Thread = (TMEM lane j =
+// value column, half hh of the key channels / of the chunk rows).
 // ============================================================================
-__device__ void state_role(const Ctx& x, const Args& p) {
+__device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v) {
   const int tid = threadIdx.x - ST_WARP0 * 32;
-  const int q = tid >> 5, lane = tid & 31;
-  const int crow = tid;                                   // key channel owned by this thread
-  const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-  uint8_t* sp = x.sm + OFF_SP;
-  uint8_t* dl = x.sm + OFF_DL;
-  const size_t sbase = (((size_t)x.n * p.n_heads + x.h) * D + crow) * D + x.j0;
-
-  float S[DV];
-  if (p.h0) {
-#pragma unroll
-    for (int m = 0; m < DV; m += 4) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(p.h0 + sbase + m));
-      S[m] = v.x; S[m + 1] = v.y; S[m + 2] = v.z; S[m + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int m = 0; m < DV; ++m) S[m] = 0.f;
-  }
-
+  const int sw = tid >> 5, lane = tid & 31;
+  const int qd = sw & 3, hh = sw >> 2;
+  const int j = 32 * qd + lane;
+  const uint32_t lb = (uint32_t)(32 * qd) << 16;
   const float* scal_all = reinterpret_cast<const float*>(x.sm + OFF_SCAL);
-  auto write_sprime = [&](const float* scal_next) {
-    const float eg = scal_next[crow];
+  const int* xflag = reinterpret_cast<const int*>(x.sm + OFF_XFLAG);
+  uint8_t* dt = x.sm + OFF_DT;
+  const size_t hbase = ((size_t)x.n * p.n_heads + x.h) * D * D;   // h0 / hT: [channel][value]
+  const int n = x.n_chunks;
+
+  // ---- prologue: the fp32 state (h0 or zeros) and cleared output accumulators
+#pragma unroll 1
+  for (int part = 0; part < 2; ++part) {
+    const int cb0 = 64 * hh + 32 * part;
+    uint32_t r[32];
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      float t[8];
+    for (int i = 0; i < 32; ++i)
+      r[i] = p.h0 ? __float_as_uint(__ldg(p.h0 + hbase + (size_t)(cb0 + i) * D + j)) : 0u;
+    tmem_st32(x.tmem + TM_S + lb + cb0, r);
+  }
+  tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
+  tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
+  tmem_st_wait();
+
+  // decay the state over chunk cc in place and write the bf16 operand S''
+  auto s_pass = [&](int cc) {
+    const float* ms = scal_all + (cc % 3) * 256;
+    const bool ex = xflag[cc % 3] != 0;
+#pragma unroll 1
+    for (int part = 0; part < 2; ++part) {
+      const int cb0 = 64 * hh + 32 * part;
+      float v[32];
+      tmem_ld32(x.tmem + TM_S + lb + cb0, v);
+      tmem_ld_wait();
+      uint32_t pk[16];
+      if (ex) {   // exact path: the operand is the undecayed state
 #pragma unroll
-      for (int e = 0; e < 8; ++e) t[e] = eg * S[ch * 8 + e];
-      *reinterpret_cast<uint4*>(sp + swz64(crow * 64 + ch * 16)) = pack8(t);
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 m4 = *reinterpret_cast<const float4*>(ms + cb0 + i);
+        v[i] *= m4.x; v[i + 1] *= m4.y; v[i + 2] *= m4.z; v[i + 3] *= m4.w;
+      }
+      if (!ex) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+      }
+      tmem_st32(x.tmem + TM_S + lb + cb0, reinterpret_cast<const uint32_t(&)[32]>(v));
+      tmem_st16(x.tmem + TM_SB + lb + cb0 / 2, pk);
     }
+    tmem_st_wait();
+    tc_fence_before();
   };
 
-  bool ok = true;
-  if (x.n_chunks > 0) {
-    ok = wait_b(x, B_TILES + 0, 0);
-    write_sprime(scal_all);
-    fence_proxy_async_smem();
-    if (named_bar_or(BAR_ST, ST_THREADS, !ok)) ok = false;
-    else if (tid == 0) mbar_arrive(&x.bars[B_SREADY]);
+  // Thread 0 issues this group's tensor-core products and the v loads. Per chunk:
+  // U (as soon as T*beta and v are there), the [O | Delta] product, then the state
+  // update and P Delta once Delta is in shared memory; the next chunk's v load goes
+  // out once the current U product is done (it precedes [O | Delta] in the pipe).
+  const bool issuer = tid == 0;
+  int u_issued = 0, v_issued = 0, v_landed = 0;
+  auto issue_u_of = [&](int cu, bool block) -> bool {
+    if (block) {
+      if (!wait_b(x, B_TB, cu & 1) || !wait_b(x, B_VFULL, cu & 1)) return false;
+    } else if (!mbar_test_wait(&x.bars[B_TB], cu & 1) || !mbar_test_wait(&x.bars[B_VFULL], cu & 1)) {
+      return true;   // not ready yet: issued later, before the chunk's [O | Delta] product
+    }
+    v_landed = cu + 1;
+    issue_u(x);
+    u_issued = cu + 1;
+    return true;
+  };
+
+  bool alive = true;
+  if (n > 0) {
+    if (issuer) {
+      issue_v(x, map_v, 0);
+      v_issued = 1;
+    }
+    alive = wait_b(x, B_TILES + 0, 0);
+    if (alive) s_pass(0);
+    named_bar_sync(BAR_ST, ST_THREADS);
+    if (issuer && alive) {
+      alive = issue_u_of(0, true) && wait_b(x, B_READY + 0, 0);
+      if (alive) issue_crit(x, 0);
+    }
   }
-  for (int c = 0; ok && c < x.n_chunks; ++c) {
-    const int s2 = c & 1, s3 = c % 3;
+  for (int c = 0; c < n; ++c) {
     const int64_t t0 = x.bos + (int64_t)c * CHUNK;
     const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
-    // ---- Delta (fp32, accumulator rows 0-63 = lanes 0-63) -> bf16 tile (warps 0-1)
-    bool okw = wait_b(x, B_ADONE, c & 1);
-    tc_fence_after();
-    if (q < 2) {
+    // ---- Delta^T (TMEM) -> bf16 tile rows j, chunk rows 32hh..32hh+31
+    alive = alive && wait_b(x, B_CRIT, c & 1);
+    if (alive) {
+      tc_fence_after();
       float v[32];
-      tmem_ld32(x.tmem + TM_C + s2 * 32 + lane_base, v);
+      tmem_ld32(x.tmem + TM_D + lb + 32 * hh, v);
       tmem_ld_wait();
-      const int r = 32 * q + lane;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch)
-        *reinterpret_cast<uint4*>(dl + swz64(r * 64 + ch * 16)) = pack8(v + ch * 8);
-    }
-    tc_fence_before();
-    fence_proxy_async_smem();
-    if (named_bar_or(BAR_ST, ST_THREADS, !okw)) break;
-    if (tid == 0) mbar_arrive(&x.bars[B_DREADY]);
-    // ---- state update: S <- e^{G_C} S + e^{G_C - G_m} (Ck^T Delta)
-    okw = wait_b(x, B_BDONE, c & 1);
-    tc_fence_after();
-    {
-      float z[32];
-      tmem_ld32(x.tmem + TM_Z + lane_base, z);
-      tmem_ld_wait();
-      const float* scal = scal_all + s3 * 384;
-      const float egc = scal[128 + crow], ecm = scal[256 + crow];
-#pragma unroll
-      for (int m = 0; m < DV; ++m) S[m] = fmaf(egc, S[m], ecm * z[m]);
-    }
-    if (c + 1 < x.n_chunks) {
-      okw = okw && wait_b(x, B_TILES + ((c + 1) & 1), ((c + 1) >> 1) & 1);
-      write_sprime(scal_all + ((c + 1) % 3) * 384);
+        *reinterpret_cast<uint4*>(dt + swz128(j * 128 + 64 * hh + 16 * ch)) = pack8(v + 8 * ch);
       fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    if (named_bar_or(BAR_ST, ST_THREADS, !okw)) break;
-    if (tid == 0) {
-      if (c + 1 < x.n_chunks) mbar_arrive(&x.bars[B_SREADY]);
-      mbar_arrive(&x.bars[B_QRFREE + s3]);
-    }
-    // ---- output epilogue (off the sequential path): accumulator rows 64-127 (warps 2-3)
-    okw = wait_b(x, B_ODONE, c & 1);
-    tc_fence_after();
-    if (q >= 2) {
-      float v[32];
-      tmem_ld32(x.tmem + TM_C + s2 * 32 + lane_base, v);
-      tmem_ld_wait();
-      const int r = 32 * (q - 2) + lane;
-      if (okw && r < L) {
-        __nv_bfloat16* orow = p.o + (size_t)(t0 + r) * x.rs + x.h * D + x.j0;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) *reinterpret_cast<uint4*>(orow + ch * 8) = pack8(v + ch * 8);
+      tc_fence_before();
+      if (issuer && c + 1 < n) {   // U(c) is done: v of the next chunk may land
+        issue_v(x, map_v, c + 1);
+        v_issued = c + 2;
       }
     }
-    tc_fence_before();
     named_bar_sync(BAR_ST, ST_THREADS);
-    if (tid == 0) mbar_arrive(&x.bars[B_DCFREE + s2]);
-  }
-  if (p.hT && !*x.abort_flag) {
+    if (issuer && alive) {
+      issue_update(x, c);
+      if (c + 1 < n) alive = issue_u_of(c + 1, false);
+    }
+    // ---- next chunk's decayed state, as soon as this chunk's update has landed
+    if (c + 1 < n) {
+      alive = alive && wait_b(x, B_ZDONE, c & 1) &&
+              wait_b(x, B_TILES + ((c + 1) & 1), ((c + 1) >> 1) & 1);
+      if (alive) {
+        tc_fence_after();
+        s_pass(c + 1);
+      }
+      named_bar_sync(BAR_ST, ST_THREADS);
+      if (issuer && alive) {
+        if (u_issued < c + 2) alive = issue_u_of(c + 1, true);
+        alive = alive && wait_b(x, B_READY + ((c + 1) & 1), ((c + 1) >> 1) & 1);
+        if (alive) issue_crit(x, c + 1);
+      }
+    }
+    // ---- output of chunk c (off the sequential path), then clear its columns
+    alive = alive && wait_b(x, B_PD, c & 1);
+    if (alive) {
+      tc_fence_after();
+      const uint32_t ro = (c & 1) ? TM_OA : TM_OB;
+      float v[32];
+      tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
+      tmem_ld_wait();
+      // lane pairs (j, j+1) swap halves: 32-bit stores of two value columns, the
+      // even lane taking the even rows and the odd lane the odd rows
+      const bool odd = lane & 1;
+      __nv_bfloat16* ocol = p.o + (size_t)t0 * x.rs + x.h * D + (j & ~1);
 #pragma unroll
-    for (int m = 0; m < DV; m += 4)
-      *reinterpret_cast<float4*>(p.hT + sbase + m) = make_float4(S[m], S[m + 1], S[m + 2], S[m + 3]);
+      for (int k = 0; k < 16; ++k) {
+        const float other = __shfl_xor_sync(0xffffffffu, odd ? v[2 * k] : v[2 * k + 1], 1);
+        const int r = 32 * hh + 2 * k + (odd ? 1 : 0);
+        const uint32_t pr = odd ? pack_bf16(other, v[2 * k + 1]) : pack_bf16(v[2 * k], other);
+        if (r < L) *reinterpret_cast<uint32_t*>(ocol + (size_t)r * x.rs) = pr;
+      }
+      tmem_st32_zero(x.tmem + ro + lb + 32 * hh);
+      tmem_st_wait();
+      tc_fence_before();
+    }
+  }
+  // ---- final state
+  if (n > 0) alive = alive && wait_b(x, B_ZDONE, (n - 1) & 1);
+  tc_fence_after();
+  if (p.hT && alive && !*x.abort_flag) {
+#pragma unroll 1
+    for (int part = 0; part < 2; ++part) {
+      const int cb0 = 64 * hh + 32 * part;
+      float v[32];
+      tmem_ld32(x.tmem + TM_S + lb + cb0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) p.hT[hbase + (size_t)(cb0 + i) * D + j] = v[i];
+    }
+  }
+  if (issuer) {
+    drain(x, B_FIN_C);
+    for (int c = v_landed; c < v_issued; ++c) settle(&x.bars[B_VFULL], c & 1);
   }
 }
 
 // ============================================================================
-// kernel
+// kernel: one CTA per (sequence, head)
 // ============================================================================
 __global__ void __launch_bounds__(THREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
@@ -989,10 +1073,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.abort_flag = reinterpret_cast<volatile int*>(x.sm + OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x.sm + OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chain = blockIdx.x / NSPLIT;
+  const int chain = blockIdx.x;
   x.n = chain / args.n_heads;
   x.h = chain % args.n_heads;
-  x.j0 = (blockIdx.x % NSPLIT) * DV;
   seq_bounds(args.cu_seqlens, x.n, args.n_seqs, args.t_total, x.bos, x.eos);
   x.n_chunks = (int)((x.eos - x.bos + CHUNK - 1) / CHUNK);
   x.rs = (size_t)args.n_heads * D;
@@ -1002,13 +1085,13 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
     *x.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == LD_WARP && lane == 0) {
+  if (threadIdx.x == 0) {
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_q);
-    prefetch_tensormap(&map_v);
     prefetch_tensormap(&map_la);
   }
-  if (warp == MC_WARP) {
+  if (warp == ST_WARP0) {
+    if (lane == 0) prefetch_tensormap(&map_v);
     tmem_alloc(tmem_slot, TM_COLS);
     tmem_relinquish();
   }
@@ -1018,21 +1101,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.tmem = *tmem_slot;
 
   if (warp < PA_WARPS) {
-    prep_a_role(x, args);
+    prep_a_role(x, args, &map_k, &map_q, &map_la);
   } else if (warp < ST_WARP0) {
     prep_b_role(x);
-  } else if (warp < LD_WARP) {
-    state_role(x, args);
-  } else if (warp == LD_WARP) {
-    if (lane == 0) load_role(x, &map_k, &map_q, &map_v, &map_la);
-  } else if (warp == MC_WARP) {
-    if (lane == 0) mma_state_role(x);
-  } else if (warp == MP_WARP) {
-    if (lane == 0) mma_prep_role(x);
+  } else {
+    state_role(x, args, &map_v);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == MC_WARP) {
+  if (warp == ST_WARP0) {
     tc_fence_after();
     tmem_dealloc(x.tmem, TM_COLS);
   }

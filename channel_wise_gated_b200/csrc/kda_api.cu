@@ -106,7 +106,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   using namespace kda::tc;
   const uint64_t cols = (uint64_t)n_heads * kda::D;
   const uint64_t rows = (uint64_t)t_total;
-  CUtensorMap mk, mq, mv, mla;
+  CUtensorMap mk, mq, mv, mla, mo;
   if (!encode_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, cols, rows, 2, 64, 64,
@@ -114,7 +114,9 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
       !encode_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, log_alpha, cols, rows, 4, 128, 64,
-                 CU_TENSOR_MAP_SWIZZLE_NONE))
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !encode_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o, cols, rows, 2, 64, 64,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
     return KDA_ERR_CUDA;
   if (cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess)
@@ -130,7 +132,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.n_heads = n_heads;
   a.t_total = t_total;
   const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
-  kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, a);
+  kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
   return launch_status();
 }
 

@@ -160,29 +160,27 @@ struct Ctx {
   size_t rs;   // elements between consecutive tokens of q/k/v/o/log_alpha
 };
 
-__device__ __forceinline__ void raise_abort(const Ctx& x) {
-  *x.abort_flag = 1;
-  flag_error(DEVERR_TIMEOUT);
-}
-
 // Bounded per-thread wait that also gives up when another role aborted. The
-// thread sleeps in the barrier (suspend hint) instead of spinning.
-__device__ __noinline__ bool wait_b_slow(const Ctx& x, uint64_t* bar, uint32_t parity) {
+// thread sleeps in the barrier (suspend hint) instead of spinning. (Out of line,
+// with scalar arguments only, so that callers keep their context in registers.)
+__device__ __noinline__ bool wait_b_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
-    if (*x.abort_flag) return false;
+    if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > WAIT_NS) {
-      raise_abort(x);
+      *abort_flag = 1;
+      flag_error(DEVERR_TIMEOUT);
       return false;
     }
   }
 }
-// Fast path inline (phase already complete), the sleeping loop out of line.
+// Fast path inline (the first try blocks until the phase completes or a short
+// hardware limit passes), the sleeping loop out of line.
 __device__ __forceinline__ bool wait_b(const Ctx& x, int b, uint32_t parity) {
   uint64_t* bar = &x.bars[b];
   if (mbar_try_wait(bar, parity)) return true;
-  return wait_b_slow(x, bar, parity);
+  return wait_b_slow(bar, parity, x.abort_flag);
 }
 
 // Global loads issued exactly where written (volatile), ahead of the barrier waits.
@@ -327,18 +325,44 @@ __device__ __forceinline__ void issue_w(const Ctx& x, int c) {
 // ============================================================================
 
 // Exact path for a chunk whose decay range is too wide for the factored Gram (kept
-// out of line: it is rare and large). Pairwise factors are evaluated one by one,
-// one channel half at a time with G staged in prep B's workspace; A goes to that
-// workspace, P to its tile, and Rk / Rq are built about the point before the chunk.
-__device__ __noinline__ bool prep_a_exact(const Ctx& x, int c, int L, uint8_t* kq, uint32_t koff,
-                                          uint32_t qoff, uint8_t* ck, const float* betas,
-                                          const float (&g2)[8][4], const float (&gc)[4]) {
+// out of line, with arguments passed by value: it is rare and large). G of this
+// thread's rows is recomputed from the (L2-resident) log-decay and the warp totals
+// still in shared memory. Pairwise factors are evaluated one by one, one channel
+// half at a time with G staged in prep B's workspace; A goes to that workspace, P
+// to its tile, and Rk / Rq are built about the point before the chunk.
+__device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, int c, int L,
+                                          uint8_t* kq, uint32_t koff, uint32_t qoff, uint8_t* ck,
+                                          const float* betas) {
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
   const int kb = lane >> 4;
   const uint32_t cbyte = (lane & 15) * 8;
   const int c0 = 4 * lane;
   float* aw = reinterpret_cast<float*>(x.sm + OFF_AW);
+  const float* wsum = reinterpret_cast<const float*>(x.sm + OFF_WSUM);
+  const float* grow = reinterpret_cast<const float*>(x.sm + OFF_GROW);
+  float g2[8][4], gc[4];
+  {
+    const int64_t t0 = x.bos + (int64_t)c * CHUNK;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int ww = 0; ww < w; ++ww)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k] += wsum[ww * 128 + c0 + k];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t t = t0 + 8 * w + j;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < x.eos) v = ldg_nc_v4(log_alpha + (size_t)t * x.rs + x.h * D + c0);
+      const float lv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[k] = fmaf(lv[k], LOG2E, acc[k]);
+        g2[j][k] = acc[k];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) gc[k] = grow[128 + c0 + k];
+  }
   // prep B must be done with chunk c-1 (its workspace) and this Ck/P slot free
   bool ok = (c < 1) || wait_b(x, B_WFREE, (c - 1) & 1);
   ok = ok && ((c < 2) || wait_b(x, B_CKFREE + (c & 1), ((c - 2) >> 1) & 1));
@@ -450,13 +474,28 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
   float* grow = reinterpret_cast<float*>(x.sm + OFF_GROW);
   int* xflag = reinterpret_cast<int*>(x.sm + OFF_XFLAG);
   const int xk = x.h * D;
-  // (thread 0) k/q loads run two chunks ahead of this role; the log-decay is
-  // prefetched into L2 three chunks ahead
+  // (thread 0) k/q loads go out as soon as their stage slot is free (its previous
+  // chunk's state product done), up to two chunks ahead of this role; the
+  // log-decay is prefetched into L2 three chunks ahead. Never blocks unless this
+  // role would otherwise wait for the tiles itself.
   int kq_issued = 0, kq_landed = 0;
+  auto push_kq = [&](int upto, bool block) {
+    while (kq_issued < x.n_chunks && kq_issued <= upto) {
+      const int cn = kq_issued;
+      if (cn >= 3) {
+        uint64_t* fb = &x.bars[B_KQFREE + cn % 3];
+        const uint32_t par = ((cn - 3) / 3) & 1;
+        if (block ? !wait_b(x, B_KQFREE + cn % 3, par) : !mbar_test_wait(fb, par)) return;
+      }
+      issue_kq(x, map_k, map_q, cn);
+      if (cn + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
+      ++kq_issued;
+    }
+  };
   if (tid == 0) {
     for (int c = 0; c < 3 && c < x.n_chunks; ++c)
       tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)c * CHUNK));
-    for (; kq_issued < 2 && kq_issued < x.n_chunks; ++kq_issued) issue_kq(x, map_k, map_q, kq_issued);
+    push_kq(1, false);
   }
 
   for (int c = 0; c < x.n_chunks; ++c) {
@@ -483,6 +522,11 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
     // role got the Ck slot of chunk c-1)
     if (tid < 64)
       betas[tid] = (t0 + tid < x.eos) ? ldg_nc_f32(p.beta + (size_t)(t0 + tid) * p.n_heads + x.h) : 0.f;
+    // loads in flight: thread 0 tops up the k/q loads (this chunk's must be out)
+    if (tid == 0) {
+      push_kq(c, true);
+      push_kq(c + 2, false);
+    }
 
     // ---- inclusive cumsum over rows, in log2 units
     {
@@ -550,7 +594,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
                          mul_bf16x2(kr.y, pack_bf16(f[2], f[3])));
       }
     } else {
-      ok = prep_a_exact(x, c, L, kq, koff, qoff, ck, betas, g2, gc);
+      ok = prep_a_exact(x, p.log_alpha, c, L, kq, koff, qoff, ck, betas);
       if (!ok) break;
     }
     // per-channel scalars and the path flag of this chunk
@@ -567,14 +611,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
     if (tid == 0) {
       mbar_arrive(&x.bars[B_TILES + (c & 1)]);
-      // k/q of chunk c+2 into the slot that chunk c-1 used (free once its state
-      // product is done), and the L2 prefetch of chunk c+3's log-decay
-      const int cn = c + 2;
-      if (cn < x.n_chunks && (cn < 3 || wait_b(x, B_KQFREE + cn % 3, ((cn - 3) / 3) & 1))) {
-        issue_kq(x, map_k, map_q, cn);
-        kq_issued = cn + 1;
-      }
-      if (c + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(c + 3) * CHUNK));
+      push_kq(c + 2, false);
     }
   }
   // never leave with copies in flight
@@ -738,13 +775,19 @@ __device__ void prep_b_role(const Ctx& x) {
       float t[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
+        float a[16];
+#pragma unroll
+        for (int i4 = 0; i4 < r; i4 += 4) {   // row r of A_qq (the pitch keeps rows 16-byte aligned)
+          const float4 a4 = *reinterpret_cast<const float4*>(&Ab[r * AW + i4]);
+          a[i4] = a4.x; a[i4 + 1] = a4.y; a[i4 + 2] = a4.z; a[i4 + 3] = a4.w;
+        }
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
         for (int i = 0; i + 1 < r; i += 2) {
-          s0 = fmaf(Ab[r * AW + i], t[i], s0);
-          s1 = fmaf(Ab[r * AW + i + 1], t[i + 1], s1);
+          s0 = fmaf(a[i], t[i], s0);
+          s1 = fmaf(a[i + 1], t[i + 1], s1);
         }
-        if (r & 1) s0 = fmaf(Ab[r * AW + r - 1], t[r - 1], s0);
+        if (r & 1) s0 = fmaf(a[r - 1], t[r - 1], s0);
         t[r] = (r == j ? 1.f : 0.f) - (s0 + s1);
       }
       __syncwarp(0x0000ffffu);
@@ -845,16 +888,14 @@ __device__ void prep_b_role(const Ctx& x) {
       issue_w(x, c);
     }
 
-    // ---- -W' readout: lane = channel ch, columns = rows r. Lane pairs (ch, ch+1) swap
-    //      halves so that each 32-bit store holds two channels of one row: the even
-    //      lane writes the even rows, the odd lane the odd rows.
+    // ---- -W' readout: lane = channel ch, columns = rows r; one 2-byte store per row
+    //      (a warp covers 64 contiguous bytes of a row)
     ok = wait_b(x, B_WDONE, c & 1);
     tc_fence_after();
     {
       const int ch = 32 * q + lane;
-      const bool odd = lane & 1;
       uint8_t* wt = kq + koff + (ch >> 6) * 16384;
-      const uint32_t cb = (uint32_t)((ch & 63) & ~1) * 2u;
+      const uint32_t cb = (uint32_t)(ch & 63) * 2u;
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         float v[32];
@@ -862,12 +903,9 @@ __device__ void prep_b_role(const Ctx& x) {
         tmem_ld_wait();
         if (ok) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float other = __shfl_xor_sync(0xffffffffu, odd ? v[2 * k] : v[2 * k + 1], 1);
-            const int r = 32 * half + 2 * k + (odd ? 1 : 0);
-            const uint32_t pr = odd ? pack_bf16(other, v[2 * k + 1]) : pack_bf16(v[2 * k], other);
-            *reinterpret_cast<uint32_t*>(wt + swz128(r * 128 + cb)) = pr;
-          }
+          for (int i = 0; i < 32; ++i)
+            *reinterpret_cast<__nv_bfloat16*>(wt + swz128((32 * half + i) * 128 + cb)) =
+                __float2bfloat16_rn(v[i]);
         }
       }
     }
@@ -886,7 +924,8 @@ __device__ void prep_b_role(const Ctx& x) {
 // state warps (12-19): the sequential pass over chunks. Thread = (TMEM lane j =
 // value column, half hh of the key channels / of the chunk rows).
 // ============================================================================
-__device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v) {
+__device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v,
+                           const CUtensorMap* map_o) {
   const int tid = threadIdx.x - ST_WARP0 * 32;
   const int sw = tid >> 5, lane = tid & 31;
   const int qd = sw & 3, hh = sw >> 2;
@@ -978,8 +1017,13 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   for (int c = 0; c < n; ++c) {
     const int64_t t0 = x.bos + (int64_t)c * CHUNK;
     const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
-    // ---- Delta^T (TMEM) -> bf16 tile rows j, chunk rows 32hh..32hh+31
+    // ---- Delta^T (TMEM) -> bf16 tile rows j, chunk rows 32hh..32hh+31. The tile
+    //      held the previous chunk's output on its way out: the store must have read it.
     alive = alive && wait_b(x, B_CRIT, c & 1);
+    if (c > 0) {
+      if (issuer) bulk_wait_read_all();
+      named_bar_sync(BAR_ST, ST_THREADS);
+    }
     if (alive) {
       tc_fence_after();
       float v[32];
@@ -1023,20 +1067,33 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       float v[32];
       tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
       tmem_ld_wait();
-      // lane pairs (j, j+1) swap halves: 32-bit stores of two value columns, the
-      // even lane taking the even rows and the odd lane the odd rows
-      const bool odd = lane & 1;
-      __nv_bfloat16* ocol = p.o + (size_t)t0 * x.rs + x.h * D + (j & ~1);
+      if (L == CHUNK) {
+        // full chunk: into the (now free) Delta^T tile in the o tile layout, then one
+        // TMA store of [64 rows][128 columns]
+        uint8_t* ot = dt + (j >> 6) * 8192;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const float other = __shfl_xor_sync(0xffffffffu, odd ? v[2 * k] : v[2 * k + 1], 1);
-        const int r = 32 * hh + 2 * k + (odd ? 1 : 0);
-        const uint32_t pr = odd ? pack_bf16(other, v[2 * k + 1]) : pack_bf16(v[2 * k], other);
-        if (r < L) *reinterpret_cast<uint32_t*>(ocol + (size_t)r * x.rs) = pr;
+        for (int i = 0; i < 32; ++i)
+          *reinterpret_cast<__nv_bfloat16*>(ot + swz128((32 * hh + i) * 128 + (j & 63) * 2)) =
+              __float2bfloat16_rn(v[i]);
+        fence_proxy_async_smem();
+      } else {
+        // ragged last chunk of a sequence: direct stores of the valid rows only
+        __nv_bfloat16* ocol = p.o + (size_t)t0 * x.rs + x.h * D + j;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (32 * hh + i < L) ocol[(size_t)(32 * hh + i) * x.rs] = __float2bfloat16_rn(v[i]);
       }
       tmem_st32_zero(x.tmem + ro + lb + 32 * hh);
       tmem_st_wait();
       tc_fence_before();
+    }
+    if (L == CHUNK) {
+      named_bar_sync(BAR_ST, ST_THREADS);
+      if (issuer && alive) {
+        tma_store_2d(map_o, dt, x.h * D, (int)t0);
+        tma_store_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);
+        bulk_commit_group();
+      }
     }
   }
   // ---- final state
@@ -1054,6 +1111,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     }
   }
   if (issuer) {
+    bulk_wait_all();
     drain(x, B_FIN_C);
     for (int c = v_landed; c < v_issued; ++c) settle(&x.bars[B_VFULL], c & 1);
   }
@@ -1065,7 +1123,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 __global__ void __launch_bounds__(THREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_la,
-                    const Args args) {
+                    const __grid_constant__ CUtensorMap map_o, const Args args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Ctx x;
   x.sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -1091,7 +1149,10 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
     prefetch_tensormap(&map_la);
   }
   if (warp == ST_WARP0) {
-    if (lane == 0) prefetch_tensormap(&map_v);
+    if (lane == 0) {
+      prefetch_tensormap(&map_v);
+      prefetch_tensormap(&map_o);
+    }
     tmem_alloc(tmem_slot, TM_COLS);
     tmem_relinquish();
   }
@@ -1105,7 +1166,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   } else if (warp < ST_WARP0) {
     prep_b_role(x);
   } else {
-    state_role(x, args, &map_v);
+    state_role(x, args, &map_v, &map_o);
   }
   tc_fence_before();
   __syncthreads();

@@ -234,9 +234,9 @@ def run_reference(args):
 
 
 def time_prefill(kda, inp, steps, warmup, ws, stream):
+    cu = None if len(inp["lens"]) == 1 else inp["cu_seqlens"]   # one sequence: no cu_seqlens
     fwd = lambda: kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
-                                h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], o=inp["o"],
-                                hT=inp["hT"])
+                                h0=inp["h0"], cu_seqlens=cu, o=inp["o"], hT=inp["hT"])
     for _ in range(warmup):
         fwd()
     torch.cuda.synchronize()
@@ -295,11 +295,13 @@ def time_e2e(kda, inp, steps, stream):
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
     d2h = o_host.numel() * o_host.element_size() + h_host.numel() * h_host.element_size()
 
+    cu = None if len(inp["lens"]) == 1 else inp["cu_seqlens"]
+
     def step():
         for n in names:
             dev[n].copy_(host[n], non_blocking=True)
         o, hT = kda.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"],
-                              h0=None, cu_seqlens=inp["cu_seqlens"], o=inp["o"], hT=inp["hT"])
+                              h0=None, cu_seqlens=cu, o=inp["o"], hT=inp["hT"])
         o_host.copy_(o, non_blocking=True)
         h_host.copy_(hT, non_blocking=True)
 

@@ -57,8 +57,9 @@ def chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, o=None, hT=Non
     beta: [T, H] fp32; h0: [N, H, 128, 128] fp32 or None; cu_seqlens: [N+1] int32
     on the device or None (one sequence). Returns (o, hT) with o like q and hT
     [N, H, 128, 128] fp32 (None if output_final_state is False).
-    ``kernel``: "auto" (tensor cores for bf16, CUDA cores for fp32) or "simt"
-    (always the fp32 CUDA-core chunk kernel).
+    ``kernel``: "auto" (tensor cores for bf16, CUDA cores for fp32; a single long
+    bf16 sequence is split in time over a workspace allocated here), "single"
+    (as "auto" but never split) or "simt" (always the fp32 CUDA-core chunk kernel).
     """
     lib = _native.load()
     if q.dim() != 3 or q.shape[2] != D:
@@ -88,12 +89,22 @@ def chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, o=None, hT=Non
         hT = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
     elif hT is not None:
         _need(hT, "hT", torch.float32, (N, H, D, D), dev)
-    fn = lib.kda_chunk_fwd_simt if kernel == "simt" else lib.kda_chunk_fwd
-    if kernel not in ("auto", "simt"):
-        raise ValueError("kernel must be 'auto' or 'simt'")
-    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
-            N, T, H, _DT[q.dtype], _ptr(o), _ptr(hT), _stream_ptr(dev))
-    _native.check(st, fn.__name__)
+    if kernel not in ("auto", "single", "simt"):
+        raise ValueError("kernel must be 'auto', 'single' or 'simt'")
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
+            N, T, H, _DT[q.dtype], _ptr(o), _ptr(hT))
+    if kernel == "simt":
+        st, name = lib.kda_chunk_fwd_simt(*args, _stream_ptr(dev)), "kda_chunk_fwd_simt"
+    else:
+        ws_bytes = 0
+        if kernel == "auto":
+            ws_bytes = lib.kda_chunk_fwd_workspace_size(N, T, H, _DT[q.dtype],
+                                                        int(cu_seqlens is not None))
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+        st = lib.kda_chunk_fwd_ws(*args, _ptr(ws), ws_bytes, _stream_ptr(dev))
+        name = "kda_chunk_fwd_ws"
+        # (the caching allocator keeps ws alive for the stream's use of it)
+    _native.check(st, name)
     return o, hT
 
 

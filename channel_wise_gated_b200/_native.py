@@ -30,6 +30,9 @@ _P, _I32, _I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
 SIGNATURES = {
     "kda_chunk_fwd": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
     "kda_chunk_fwd_simt": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
+    "kda_chunk_fwd_ws": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P,
+                         ctypes.c_size_t, _P],
+    "kda_chunk_fwd_workspace_size": [_I32, _I64, _I32, ctypes.c_int, ctypes.c_int],
     "kda_decode_step": [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, ctypes.c_int, ctypes.c_int, _P],
     "kda_device_status": [_P],
     "kda_status_string": [ctypes.c_int],
@@ -57,7 +60,8 @@ def load(path: str = LIB_PATH):
     for name, argtypes in SIGNATURES.items():
         fn = getattr(lib, name)
         fn.argtypes = argtypes
-        fn.restype = ctypes.c_char_p if name == "kda_status_string" else ctypes.c_int
+        fn.restype = {"kda_status_string": ctypes.c_char_p,
+                      "kda_chunk_fwd_workspace_size": ctypes.c_size_t}.get(name, ctypes.c_int)
     _lib = lib
     return lib
 

@@ -13,6 +13,7 @@
 #include "kda_chunk_tc.cuh"
 #include "kda_common.cuh"
 #include "kda_decode.cuh"
+#include "kda_segment.cuh"
 
 namespace {
 
@@ -100,9 +101,35 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Time split of one long sequence (see the chunk kernel's plans): the number of
+// segments n (0 = none) for H heads and n_chunks chunks. Both passes must fit one
+// wave of the machine (H (2n - 3) CTAs for the state pass, H n for the outputs),
+// and each segment keeps at least MIN_SEG_CHUNKS chunks; the split pays off from
+// n = 3 (two passes over n segments each: n / 2 of the single-pass time).
+constexpr int MIN_SEG_CHUNKS = 16;
+constexpr int MAX_SEGMENTS = 64;
+
+int segment_count(int32_t n_heads, int64_t n_chunks) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  int best = 0;
+  for (int n = 3; n <= MAX_SEGMENTS; ++n) {
+    if ((int64_t)n_heads * (2 * n - 3) > sms || n_chunks < (int64_t)n * MIN_SEG_CHUNKS) break;
+    best = n;
+  }
+  return best;
+}
+
+size_t segment_workspace_bytes(int n_seg, int32_t n_heads) {
+  return n_seg >= 3 ? (size_t)kda::seg::slots(n_seg) * n_heads * kda::D * kda::D * sizeof(float) : 0;
+}
+
 int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
                     const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
-                    int64_t t_total, int32_t n_heads, void* o, float* hT, cudaStream_t stream) {
+                    int64_t t_total, int32_t n_heads, void* o, float* hT, int n_seg,
+                    float* seg_states, cudaStream_t stream) {
   using namespace kda::tc;
   const uint64_t cols = (uint64_t)n_heads * kda::D;
   const uint64_t rows = (uint64_t)t_total;
@@ -131,9 +158,53 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.n_seqs = n_seqs;
   a.n_heads = n_heads;
   a.t_total = t_total;
-  const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
-  kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
+  a.plan = PLAN_SEQ;
+  a.n_seg = 0;
+  a.seg_chunks = 0;
+  a.seg_states = nullptr;
+  if (n_seg < 3 || seg_states == nullptr) {
+    const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
+    kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
+    return launch_status();
+  }
+  // time split: segment states, the scan over segments, then the outputs
+  const int64_t n_chunks = (t_total + kda::CHUNK - 1) / kda::CHUNK;
+  a.n_seg = n_seg;
+  a.seg_chunks = (int)((n_chunks + n_seg - 1) / n_seg);
+  a.seg_states = seg_states;
+  a.plan = PLAN_STATES;
+  kda_chunk_tc_kernel<<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
+      mk, mq, mv, mla, mo, a);
+  if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
+  if (n_seg > 2) {
+    if (cudaFuncSetAttribute(kda::seg::kda_segment_scan_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kda::seg::SCAN_SMEM) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    kda::seg::kda_segment_scan_kernel<<<(unsigned)n_heads, kda::seg::SCAN_THREADS,
+                                         kda::seg::SCAN_SMEM, stream>>>(seg_states, n_heads, n_seg);
+    if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
+  }
+  a.plan = PLAN_OUTPUTS;
+  kda_chunk_tc_kernel<<<(unsigned)(n_heads * n_seg), THREADS, SMEM_BYTES, stream>>>(
+      mk, mq, mv, mla, mo, a);
   return launch_status();
+}
+
+// Whether a call takes the tensor-core path and, if so, how many segments it splits into.
+bool use_tc(const int32_t* cu_seqlens, int32_t n_seqs, int64_t t_total, int32_t n_heads,
+            kda_dtype qkv_dtype) {
+  (void)cu_seqlens;
+  // bf16 inputs run on the tensor-core kernel; its TMA boxes span 64 tokens, so
+  // inputs shorter than one chunk (and fp32 inputs) take the CUDA-core kernel.
+  return qkv_dtype == KDA_BF16 && t_total >= kda::CHUNK &&
+         t_total < (int64_t)INT32_MAX - 4 * kda::CHUNK && (int64_t)n_seqs * n_heads < (int64_t)INT32_MAX;
+}
+int plan_segments(const int32_t* cu_seqlens, int32_t n_seqs, int64_t t_total, int32_t n_heads,
+                  kda_dtype qkv_dtype) {
+  if (!use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype) || cu_seqlens != nullptr || n_seqs != 1)
+    return 0;
+  return segment_count(n_heads, (t_total + kda::CHUNK - 1) / kda::CHUNK);
 }
 
 template <typename TQ, typename TG>
@@ -166,15 +237,33 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_
                   const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                   int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
                   cudaStream_t stream) {
+  return kda_chunk_fwd_ws(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                          qkv_dtype, o, hT, nullptr, 0, stream);
+}
+
+size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_heads,
+                                    kda_dtype qkv_dtype, int has_cu_seqlens) {
+  if (n_heads <= 0 || n_seqs <= 0 || t_total < 0) return 0;
+  static const int32_t dummy = 0;
+  const int n_seg = plan_segments(has_cu_seqlens ? &dummy : nullptr, n_seqs, t_total, n_heads,
+                                  qkv_dtype);
+  return segment_workspace_bytes(n_seg, n_heads);
+}
+
+int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* log_alpha,
+                     const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                     int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
+                     void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                                qkv_dtype, o, hT);
   if (st != KDA_OK) return st;
-  // bf16 inputs run on the tensor-core kernel; its TMA boxes span 64 tokens, so
-  // inputs shorter than one chunk (and fp32 inputs) take the CUDA-core kernel.
-  if (qkv_dtype == KDA_BF16 && t_total >= kda::CHUNK && t_total < (int64_t)INT32_MAX - 4 * kda::CHUNK &&
-      (int64_t)n_seqs * n_heads < (int64_t)INT32_MAX)
+  if (workspace && !aligned16(workspace)) return KDA_ERR_ALIGN;
+  if (use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype)) {
+    int n_seg = plan_segments(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype);
+    if (workspace == nullptr || workspace_bytes < segment_workspace_bytes(n_seg, n_heads)) n_seg = 0;
     return launch_chunk_tc(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads, o,
-                           hT, stream);
+                           hT, n_seg, static_cast<float*>(workspace), stream);
+  }
   return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                              qkv_dtype, o, hT, stream);
 }

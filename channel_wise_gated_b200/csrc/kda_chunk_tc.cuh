@@ -138,6 +138,20 @@ enum : int {
 };
 static_assert(NUM_BARS <= NBARS, "barrier slots");
 
+// Work plans. PLAN_SEQ: one CTA per (sequence of cu_seqlens, head). The time split
+// of one long sequence into n_seg segments of seg_chunks chunks (the last takes the
+// rest) runs as PLAN_STATES, then the segment scan, then PLAN_OUTPUTS:
+//   PLAN_STATES (grid H x (2 n_seg - 3)), slot s of head h:
+//     s = 0                 segment 0 from the caller's h0: the state entering segment 1
+//     s = 1 .. n_seg-2      segment s from a zero state (R_s)
+//     s = n_seg-1 .. 2n-4   segment s-(n_seg-2) from the identity with v = 0 (its
+//                           transition M_s: S_end = M_s S_start + R_s)
+//   and each writes its final state to seg_states[s][h]; no output.
+//   PLAN_OUTPUTS (grid H x n_seg): segment j from its true entering state (the
+//     caller's h0, slot 0, or the scan's result in slot 2 n_seg - 5 + j), writing o,
+//     and the caller's hT for the last segment.
+enum : int { PLAN_SEQ = 0, PLAN_STATES = 1, PLAN_OUTPUTS = 2 };
+
 struct Args {
   const float* log_alpha;
   const float* beta;
@@ -148,6 +162,10 @@ struct Args {
   int n_seqs;
   int n_heads;
   int64_t t_total;
+  int plan;
+  int n_seg;
+  int seg_chunks;
+  float* seg_states;   // [3 n_seg - 5][H][128][128]
 };
 
 struct Ctx {
@@ -155,9 +173,14 @@ struct Ctx {
   uint64_t* bars;
   volatile int* abort_flag;
   uint32_t tmem;
-  int n, h, n_chunks;
+  int h, n_chunks;
   int64_t bos, eos;
-  size_t rs;   // elements between consecutive tokens of q/k/v/o/log_alpha
+  size_t rs;          // elements between consecutive tokens of q/k/v/o/log_alpha
+  const float* h0;    // this CTA's entering state [channel][value], or null (zeros)
+  float* hT;          // where its final state goes, or null
+  bool h0_identity;   // entering state = I (transition of a segment)
+  bool v_zero;        // v taken as zero (no loads)
+  bool write_o;       // store the output
 };
 
 // Bounded per-thread wait that also gives up when another role aborted. The
@@ -246,6 +269,10 @@ __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* map_v, 
   const int xk = x.h * D;
   const int y = (int)(x.bos + (int64_t)c * CHUNK);
   uint64_t* full = &x.bars[B_VFULL];
+  if (x.v_zero) {   // the v tile stays zero: complete the phase without a copy
+    mbar_arrive(full);
+    return;
+  }
   mbar_arrive_expect_tx(full, 2 * 8192);
   tma_load_2d(x.sm + OFF_V, map_v, xk, y, full);
   tma_load_2d(x.sm + OFF_V + 8192, map_v, xk + 64, y, full);
@@ -934,7 +961,6 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   const float* scal_all = reinterpret_cast<const float*>(x.sm + OFF_SCAL);
   const int* xflag = reinterpret_cast<const int*>(x.sm + OFF_XFLAG);
   uint8_t* dt = x.sm + OFF_DT;
-  const size_t hbase = ((size_t)x.n * p.n_heads + x.h) * D * D;   // h0 / hT: [channel][value]
   const int n = x.n_chunks;
 
   // ---- prologue: the fp32 state (h0 or zeros) and cleared output accumulators
@@ -944,12 +970,18 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     uint32_t r[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i)
-      r[i] = p.h0 ? __float_as_uint(__ldg(p.h0 + hbase + (size_t)(cb0 + i) * D + j)) : 0u;
+      r[i] = x.h0 ? __float_as_uint(__ldg(x.h0 + (size_t)(cb0 + i) * D + j))
+                  : (x.h0_identity && cb0 + i == j ? 0x3F800000u : 0u);
     tmem_st32(x.tmem + TM_S + lb + cb0, r);
   }
   tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
   tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
   tmem_st_wait();
+  if (x.v_zero) {   // a zero v tile for every chunk (U = 0)
+    for (int i = tid; i < 1024; i += ST_THREADS)
+      *reinterpret_cast<uint4*>(x.sm + OFF_V + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
 
   // decay the state over chunk cc in place and write the bf16 operand S''
   auto s_pass = [&](int cc) {
@@ -1067,7 +1099,9 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       float v[32];
       tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
       tmem_ld_wait();
-      if (L == CHUNK) {
+      if (!x.write_o) {
+        // (segment state pass: no output)
+      } else if (L == CHUNK) {
         // full chunk: into the (now free) Delta^T tile in the o tile layout, then one
         // TMA store of [64 rows][128 columns]
         uint8_t* ot = dt + (j >> 6) * 8192;
@@ -1087,7 +1121,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       tmem_st_wait();
       tc_fence_before();
     }
-    if (L == CHUNK) {
+    if (L == CHUNK && x.write_o) {
       named_bar_sync(BAR_ST, ST_THREADS);
       if (issuer && alive) {
         tma_store_2d(map_o, dt, x.h * D, (int)t0);
@@ -1099,7 +1133,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   // ---- final state
   if (n > 0) alive = alive && wait_b(x, B_ZDONE, (n - 1) & 1);
   tc_fence_after();
-  if (p.hT && alive && !*x.abort_flag) {
+  if (x.hT && alive && !*x.abort_flag) {
 #pragma unroll 1
     for (int part = 0; part < 2; ++part) {
       const int cb0 = 64 * hh + 32 * part;
@@ -1107,7 +1141,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       tmem_ld32(x.tmem + TM_S + lb + cb0, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) p.hT[hbase + (size_t)(cb0 + i) * D + j] = v[i];
+      for (int i = 0; i < 32; ++i) x.hT[(size_t)(cb0 + i) * D + j] = v[i];
     }
   }
   if (issuer) {
@@ -1131,12 +1165,48 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.abort_flag = reinterpret_cast<volatile int*>(x.sm + OFF_MISC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x.sm + OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chain = blockIdx.x;
-  x.n = chain / args.n_heads;
-  x.h = chain % args.n_heads;
-  seq_bounds(args.cu_seqlens, x.n, args.n_seqs, args.t_total, x.bos, x.eos);
+  const int H = args.n_heads;
+  const int slot = blockIdx.x / H;
+  x.h = blockIdx.x % H;
+  x.rs = (size_t)H * D;
+  x.h0_identity = false;
+  x.v_zero = false;
+  x.write_o = true;
+  const size_t state_elems = (size_t)D * D;
+  if (args.plan == PLAN_SEQ) {
+    seq_bounds(args.cu_seqlens, slot, args.n_seqs, args.t_total, x.bos, x.eos);
+    const size_t sidx = ((size_t)slot * H + x.h) * state_elems;
+    x.h0 = args.h0 ? args.h0 + sidx : nullptr;
+    x.hT = args.hT ? args.hT + sidx : nullptr;
+  } else {
+    const int ns = args.n_seg;
+    int seg;
+    if (args.plan == PLAN_STATES) {
+      x.write_o = false;
+      x.h0 = nullptr;
+      if (slot == 0) {
+        seg = 0;
+        x.h0 = args.h0 ? args.h0 + (size_t)x.h * state_elems : nullptr;
+      } else if (slot <= ns - 2) {
+        seg = slot;
+      } else {
+        seg = slot - (ns - 2);
+        x.h0_identity = true;
+        x.v_zero = true;
+      }
+      x.hT = args.seg_states + ((size_t)slot * H + x.h) * state_elems;
+    } else {
+      seg = slot;
+      if (seg == 0)
+        x.h0 = args.h0 ? args.h0 + (size_t)x.h * state_elems : nullptr;
+      else
+        x.h0 = args.seg_states + ((size_t)(seg == 1 ? 0 : 2 * ns - 5 + seg) * H + x.h) * state_elems;
+      x.hT = (seg == ns - 1 && args.hT) ? args.hT + (size_t)x.h * state_elems : nullptr;
+    }
+    x.bos = (int64_t)seg * args.seg_chunks * CHUNK;
+    x.eos = (seg == ns - 1) ? args.t_total : x.bos + (int64_t)args.seg_chunks * CHUNK;
+  }
   x.n_chunks = (int)((x.eos - x.bos + CHUNK - 1) / CHUNK);
-  x.rs = (size_t)args.n_heads * D;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(&x.bars[i], 1);

@@ -1,0 +1,78 @@
+// Time split of one long sequence: composition of the segments' state maps.
+//
+// Every step of the recurrence (Kimi Linear summary, section 3) is affine in the
+// state, so a segment of chunks maps its entering state S to M S + R, with M the
+// product of its per-token transitions (I - beta k k^T) Diag(alpha) and R its final
+// state from a zero start. The chunk kernel's state pass computes, per head, the
+// exact state entering segment 1 (slot 0), R_s (slots 1 .. n-2) and M_s (slots
+// n-1 .. 2n-4, the final state from the identity with v = 0). This kernel then
+// walks the segments in order,
+//     S_j = M_{j-1} S_{j-1} + R_{j-1},   j = 2 .. n-1,
+// writing S_j to slot 2n-5+j, all in fp32. One CTA per head; n-2 products of
+// 128 x 128 matrices, a few microseconds in all.
+#pragma once
+
+#include "kda_common.cuh"
+
+namespace kda {
+namespace seg {
+
+constexpr int SCAN_THREADS = 256;
+constexpr int SP = D + 4;   // smem pitch of the row-major copies (keeps float4 rows aligned)
+constexpr size_t SCAN_SMEM = 2 * (size_t)D * SP * sizeof(float);
+
+// Slots of the segment-state buffer [slots][H][128][128] (see the chunk kernel's plans).
+__host__ __device__ constexpr int slots(int n_seg) { return 3 * n_seg - 5; }
+
+__global__ void __launch_bounds__(SCAN_THREADS)
+kda_segment_scan_kernel(float* __restrict__ states, int n_heads, int n_seg) {
+  extern __shared__ __align__(16) float sm[];
+  float* Ms = sm;             // M_{j-1}, row-major, pitch SP
+  float* Ss = sm + D * SP;    // S_{j-1}
+  const int h = blockIdx.x, tid = threadIdx.x;
+  const size_t E = (size_t)D * D;
+  auto slot = [&](int s) { return states + ((size_t)s * n_heads + h) * E; };
+  // thread tile: rows r0..r0+7, columns c0..c0+7 of the 128 x 128 result
+  const int r0 = 8 * (tid >> 4), c0 = 8 * (tid & 15);
+  for (int j = 2; j < n_seg; ++j) {
+    const float* M = slot(n_seg - 3 + j);                    // M_{j-1}
+    const float* S = slot(j == 2 ? 0 : 2 * n_seg - 6 + j);   // S_{j-1}
+    const float* R = slot(j - 1);                            // R_{j-1}
+    float* out = slot(2 * n_seg - 5 + j);                    // S_j
+    for (int i = tid; i < D * D / 4; i += SCAN_THREADS) {
+      const int r = (4 * i) / D, c = (4 * i) % D;
+      *reinterpret_cast<float4*>(&Ms[r * SP + c]) = reinterpret_cast<const float4*>(M)[i];
+      *reinterpret_cast<float4*>(&Ss[r * SP + c]) = reinterpret_cast<const float4*>(S)[i];
+    }
+    __syncthreads();
+    float acc[8][8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < D; ++k) {
+      float av[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) av[a] = Ms[(r0 + a) * SP + k];
+      const float4 b0 = *reinterpret_cast<const float4*>(&Ss[k * SP + c0]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Ss[k * SP + c0 + 4]);
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
+    }
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const size_t e = (size_t)(r0 + a) * D + c0 + b;
+        out[e] = acc[a][b] + R[e];
+      }
+    __syncthreads();
+  }
+}
+
+}  // namespace seg
+}  // namespace kda

@@ -27,7 +27,8 @@
  * Conventions for every entry point:
  *   - Head dimension is fixed: d_k = d_v = 128.
  *   - Every pointer is a DEVICE pointer owned by the caller. The library
- *     allocates no device memory and keeps no per-call state.
+ *     allocates no device memory and keeps no per-call state (scratch, where an
+ *     entry point can use it, is a caller-provided workspace).
  *   - Calls are asynchronous and ordered on `stream`. A return of KDA_OK means
  *     "arguments validated and kernel launched"; device-side problems (bad
  *     cu_seqlens contents) are reported later by kda_device_status().
@@ -38,6 +39,7 @@
 #ifndef KDA_B200_H
 #define KDA_B200_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -92,6 +94,41 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_
                   const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                   int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
                   cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_ws - kda_chunk_fwd with a caller-provided workspace, which lets a
+ * single long bf16 sequence (cu_seqlens == NULL, n_seqs == 1) be split in time.
+ *
+ * Every step of the recurrence is affine in the state, so a run of chunks maps
+ * its entering state S to M S + R (M: product of the per-token transitions,
+ * R: the final state from a zero start). With the time split the sequence is cut
+ * into n segments (n >= 3, chosen so that both passes fit one wave of the GPU):
+ * a first pass computes, in parallel, the exact state entering segment 1 and
+ * (R_s, M_s) of the middle segments; a scan composes them into the state entering
+ * every segment; a second pass runs all segments in parallel from those states
+ * and writes o and hT. The result is the same recurrence (exact in real
+ * arithmetic; fp32 state throughout, bf16 MMA operands as in kda_chunk_fwd).
+ *
+ * Arguments: as kda_chunk_fwd, plus
+ *   workspace        16-byte aligned device scratch, or NULL
+ *   workspace_bytes  its size; the split runs only when it is at least
+ *                    kda_chunk_fwd_workspace_size(...) > 0, otherwise the call is
+ *                    exactly kda_chunk_fwd (single pass)
+ * The workspace must stay untouched until the stream has passed the call.
+ * Returns KDA_OK or a negative kda_status (KDA_ERR_ALIGN for a misaligned workspace).
+ */
+int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* log_alpha,
+                     const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                     int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
+                     void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_workspace_size - bytes of workspace kda_chunk_fwd_ws would use for
+ * these sizes on the current device (0: no time split applies). has_cu_seqlens is
+ * nonzero when the call will pass a cu_seqlens array (then no split applies).
+ */
+size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_heads,
+                                    kda_dtype qkv_dtype, int has_cu_seqlens);
 
 /*
  * kda_chunk_fwd_simt - the same operation as kda_chunk_fwd, always on the fp32

@@ -72,6 +72,23 @@ def test_chunk_validation(lib):
     assert _chunk(lib, n=2, cu=None) == _native.KDA_ERR_SEQLENS
     assert lib.kda_chunk_fwd_simt(None, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2,
                                   _native.KDA_F32, FAKE, None, None) == _native.KDA_ERR_NULL
+    # the workspace entry point: same validation, plus an aligned workspace
+    ws = lib.kda_chunk_fwd_ws
+    assert ws(None, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, _native.KDA_BF16, FAKE, None,
+              FAKE, 1 << 20, None) == _native.KDA_ERR_NULL
+    assert ws(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, _native.KDA_BF16, FAKE, None,
+              FAKE + 8, 1 << 20, None) == _native.KDA_ERR_ALIGN
+
+
+def test_workspace_size_queries(lib):
+    size = lib.kda_chunk_fwd_workspace_size
+    bf, f32 = _native.KDA_BF16, _native.KDA_F32
+    # no time split for fp32, packed batches, short sequences or bad sizes
+    assert size(1, 1 << 20, 32, f32, 0) == 0
+    assert size(1, 1 << 20, 32, bf, 1) == 0
+    assert size(1, 64 * 16, 32, bf, 0) == 0
+    assert size(0, 1 << 20, 32, bf, 0) == 0
+    assert size(1, 1 << 20, 0, bf, 0) == 0
 
 
 def test_decode_validation(lib):

@@ -55,8 +55,20 @@ def _oracle(inp, heads=None):
 
 
 def _run(kda, inp, kernel="auto"):
+    # a single sequence goes in without cu_seqlens, as bench.py passes it (this is
+    # what lets a long one be split in time)
+    cu = None if len(inp["lens"]) == 1 else inp["cu_seqlens"]
     return kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
-                         h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], kernel=kernel)
+                         h0=inp["h0"], cu_seqlens=cu, kernel=kernel)
+
+
+def _split_segments(kda, T, H):
+    """Segments the time split uses for one bf16 sequence (0: no split)."""
+    ws = kda._native.load().kda_chunk_fwd_workspace_size(1, T, H, kda._native.KDA_BF16, 0)
+    if ws == 0:
+        return 0
+    slots = ws // (H * 128 * 128 * 4)
+    return (slots + 5) // 3
 
 
 @pytest.mark.parametrize("kernel", ["auto", "simt"])
@@ -179,6 +191,54 @@ def test_strong_decay_stress(kda, dtype):
     tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
     assert rel_err(o, o_ref) <= tol
     assert rel_err(hT, h_ref) <= max(tol, 1e-30)
+
+
+def test_time_split_32_heads_ragged(kda):
+    """One long sequence split in time (3 segments at 32 heads), random h0, ragged tail."""
+    T, H = 64 * 60 + 37, 32
+    assert _split_segments(kda, T, H) == 3
+    inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 3.0, True, seed=81,
+                                  device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    assert rel_err(o, o_ref) <= TOL_BF16
+    assert rel_err(hT, h_ref) <= TOL_BF16
+
+
+def test_time_split_16_heads_mixed_decay(kda):
+    """16 heads split into 6 segments; strong-decay chunks put exact-path chunks into
+    every pass (the transition runs start from the identity with v = 0)."""
+    T, H = 64 * 100 + 5, 16
+    assert _split_segments(kda, T, H) == 6
+    inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 3.0, True, seed=82,
+                                  device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(83)
+    la = inp["log_alpha"]
+    for c in (3, 17, 18, 40, 41, 70, 99):
+        rows = slice(64 * c, 64 * c + 64)
+        x = torch.randn(la[rows].shape, generator=g, device="cuda") - 5.0
+        la[rows] = torch.nn.functional.logsigmoid(x)
+    # and slow decay elsewhere, so that segment transitions do not vanish
+    slow = torch.ones(T, dtype=torch.bool, device="cuda")
+    for c in (3, 17, 18, 40, 41, 70, 99):
+        slow[64 * c:64 * c + 64] = False
+    la[slow] *= 0.05
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    assert rel_err(o, o_ref) <= TOL_BF16
+    assert rel_err(hT, h_ref) <= TOL_BF16
+
+
+def test_time_split_equals_single_pass(kda):
+    """The split and the single pass compute the same recurrence."""
+    T, H = 64 * 64, 32
+    inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 3.0, True, seed=84,
+                                  device="cuda")
+    o_s, h_s = _run(kda, inp, kernel="auto")
+    o_1, h_1 = _run(kda, inp, kernel="single")
+    assert _split_segments(kda, T, H) == 3
+    assert rel_err(o_s, o_1.double().cpu().numpy()) <= TOL_BF16
+    assert rel_err(h_s, h_1.double().cpu().numpy()) <= TOL_BF16
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])

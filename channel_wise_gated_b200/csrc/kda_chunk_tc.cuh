@@ -947,6 +947,49 @@ __device__ void prep_b_role(const Ctx& x) {
   if (tid == 0) drain(x, B_FIN_P);
 }
 
+// ---- cold paths of the state warps, out of line with scalar arguments (they run
+//      once per CTA or once per sequence and would otherwise cost the hot loop
+//      registers). Thread = TMEM lane j of its warp's quarter (lane_addr), 64
+//      channels (or 32 rows) starting at cb.
+
+// the entering state (h0, the identity, or zeros) into the fp32 master, [channel][value]
+__device__ __noinline__ void st_load_state(uint32_t lane_addr, const float* h0, bool identity, int j,
+                                           int cb) {
+#pragma unroll 1
+  for (int part = 0; part < 2; ++part) {
+    const int cb0 = cb + 32 * part;
+    uint32_t r[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      r[i] = h0 ? __float_as_uint(__ldg(h0 + (size_t)(cb0 + i) * D + j))
+                : (identity && cb0 + i == j ? 0x3F800000u : 0u);
+    tmem_st32(lane_addr + cb0, r);
+  }
+  tmem_st_wait();
+}
+// the final state out of the fp32 master
+__device__ __noinline__ void st_store_state(uint32_t lane_addr, float* hT, int j, int cb) {
+#pragma unroll 1
+  for (int part = 0; part < 2; ++part) {
+    const int cb0 = cb + 32 * part;
+    float v[32];
+    tmem_ld32(lane_addr + cb0, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) hT[(size_t)(cb0 + i) * D + j] = v[i];
+  }
+}
+// output rows r0.. of a ragged last chunk (the valid rows < L only), direct stores
+__device__ __noinline__ void st_store_ragged(uint32_t lane_addr, __nv_bfloat16* ocol, size_t rs,
+                                             int r0, int L) {
+  float v[32];
+  tmem_ld32(lane_addr, v);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if (r0 + i < L) ocol[(size_t)(r0 + i) * rs] = __float2bfloat16_rn(v[i]);
+}
+
 // ============================================================================
 // state warps (12-19): the sequential pass over chunks. Thread = (TMEM lane j =
 // value column, half hh of the key channels / of the chunk rows).
@@ -963,17 +1006,8 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   uint8_t* dt = x.sm + OFF_DT;
   const int n = x.n_chunks;
 
-  // ---- prologue: the fp32 state (h0 or zeros) and cleared output accumulators
-#pragma unroll 1
-  for (int part = 0; part < 2; ++part) {
-    const int cb0 = 64 * hh + 32 * part;
-    uint32_t r[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      r[i] = x.h0 ? __float_as_uint(__ldg(x.h0 + (size_t)(cb0 + i) * D + j))
-                  : (x.h0_identity && cb0 + i == j ? 0x3F800000u : 0u);
-    tmem_st32(x.tmem + TM_S + lb + cb0, r);
-  }
+  // ---- prologue: the fp32 state (h0, identity or zeros) and cleared output accumulators
+  st_load_state(x.tmem + TM_S + lb, x.h0, x.h0_identity, j, 64 * hh);
   tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
   tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
   tmem_st_wait();
@@ -1096,14 +1130,14 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     if (alive) {
       tc_fence_after();
       const uint32_t ro = (c & 1) ? TM_OA : TM_OB;
-      float v[32];
-      tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
-      tmem_ld_wait();
       if (!x.write_o) {
         // (segment state pass: no output)
       } else if (L == CHUNK) {
         // full chunk: into the (now free) Delta^T tile in the o tile layout, then one
         // TMA store of [64 rows][128 columns]
+        float v[32];
+        tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
+        tmem_ld_wait();
         uint8_t* ot = dt + (j >> 6) * 8192;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
@@ -1112,10 +1146,8 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         fence_proxy_async_smem();
       } else {
         // ragged last chunk of a sequence: direct stores of the valid rows only
-        __nv_bfloat16* ocol = p.o + (size_t)t0 * x.rs + x.h * D + j;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (32 * hh + i < L) ocol[(size_t)(32 * hh + i) * x.rs] = __float2bfloat16_rn(v[i]);
+        st_store_ragged(x.tmem + ro + lb + 32 * hh, p.o + (size_t)t0 * x.rs + x.h * D + j, x.rs,
+                        32 * hh, L);
       }
       tmem_st32_zero(x.tmem + ro + lb + 32 * hh);
       tmem_st_wait();
@@ -1133,17 +1165,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   // ---- final state
   if (n > 0) alive = alive && wait_b(x, B_ZDONE, (n - 1) & 1);
   tc_fence_after();
-  if (x.hT && alive && !*x.abort_flag) {
-#pragma unroll 1
-    for (int part = 0; part < 2; ++part) {
-      const int cb0 = 64 * hh + 32 * part;
-      float v[32];
-      tmem_ld32(x.tmem + TM_S + lb + cb0, v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x.hT[(size_t)(cb0 + i) * D + j] = v[i];
-    }
-  }
+  if (x.hT && alive && !*x.abort_flag) st_store_state(x.tmem + TM_S + lb, x.hT, j, 64 * hh);
   if (issuer) {
     bulk_wait_all();
     drain(x, B_FIN_C);

@@ -356,6 +356,11 @@ def main():
     inp["hT"] = torch.empty((N, H, D, D), dtype=torch.float32, device="cuda")
     step_bytes = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + N * H * STATE_BYTES * (
         2 if inp["h0"] is not None else 1)
+    # one prefill call = one launch of the chunk kernel, or, for one long sequence
+    # split in time, its state pass + the segment scan + its output pass
+    split = N == 1 and kda._native.load().kda_chunk_fwd_workspace_size(
+        1, T, H, kda._native.KDA_BF16, 0) > 0
+    launches_per_call = 3 if split else 1
 
     with ClockSampler(local) as clk:
         total_ms, per_launch = time_prefill(kda, inp, args.steps, args.warmup, ws, stream)
@@ -408,11 +413,14 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": None,
                          "peak_kind": peak_kind,
-                         "algorithmic_bytes_per_launch": step_bytes,
-                         "avg_launch_ms": avg_launch_ms},
+                         "kernel": "kda_chunk_tc_kernel",
+                         "unit_of_work": ("one prefill call (state pass + segment scan + "
+                                          "output pass)" if split else "one launch"),
+                         "algorithmic_bytes_per_call": step_bytes,
+                         "avg_call_ms": avg_launch_ms},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * launches_per_call,
             "clocks": clocks,
             "decode": {"workload": dcfg.name, "steps": args.decode_steps,
                        "us_per_step": dec_step_us, "GBps": dec_gbs,

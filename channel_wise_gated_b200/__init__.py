@@ -58,8 +58,10 @@ def chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, o=None, hT=Non
     on the device or None (one sequence). Returns (o, hT) with o like q and hT
     [N, H, 128, 128] fp32 (None if output_final_state is False).
     ``kernel``: "auto" (tensor cores for bf16, CUDA cores for fp32; a single long
-    bf16 sequence is split in time over a workspace allocated here), "single"
-    (as "auto" but never split) or "simt" (always the fp32 CUDA-core chunk kernel).
+    bf16 sequence is split in time over a workspace allocated here), "static" (as
+    "auto", with the library's module-resident scratch instead: no allocation),
+    "single" (as "auto" but never split) or "simt" (always the fp32 CUDA-core chunk
+    kernel).
     """
     lib = _native.load()
     if q.dim() != 3 or q.shape[2] != D:
@@ -89,12 +91,14 @@ def chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, o=None, hT=Non
         hT = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
     elif hT is not None:
         _need(hT, "hT", torch.float32, (N, H, D, D), dev)
-    if kernel not in ("auto", "single", "simt"):
-        raise ValueError("kernel must be 'auto', 'single' or 'simt'")
+    if kernel not in ("auto", "static", "single", "simt"):
+        raise ValueError("kernel must be 'auto', 'static', 'single' or 'simt'")
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
             N, T, H, _DT[q.dtype], _ptr(o), _ptr(hT))
     if kernel == "simt":
         st, name = lib.kda_chunk_fwd_simt(*args, _stream_ptr(dev)), "kda_chunk_fwd_simt"
+    elif kernel == "static":
+        st, name = lib.kda_chunk_fwd_static(*args, _stream_ptr(dev)), "kda_chunk_fwd_static"
     else:
         ws_bytes = 0
         if kernel == "auto":

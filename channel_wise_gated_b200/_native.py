@@ -33,6 +33,7 @@ SIGNATURES = {
     "kda_chunk_fwd_ws": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P,
                          ctypes.c_size_t, _P],
     "kda_chunk_fwd_workspace_size": [_I32, _I64, _I32, ctypes.c_int, ctypes.c_int],
+    "kda_chunk_fwd_static": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
     "kda_decode_step": [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, ctypes.c_int, ctypes.c_int, _P],
     "kda_device_status": [_P],
     "kda_status_string": [ctypes.c_int],

@@ -15,6 +15,12 @@
 #include "kda_decode.cuh"
 #include "kda_segment.cuh"
 
+// Scratch of kda_chunk_fwd_static: module-resident device memory (no allocation at
+// call time), large enough for the time split of any head count on a 148-SM part
+// (slots x heads <= 3 x 74 + 5, 64 KiB each).
+constexpr size_t STATIC_SCRATCH_BYTES = (size_t)16 << 20;
+static __device__ __align__(256) unsigned char g_kda_static_scratch[STATIC_SCRATCH_BYTES];
+
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -266,6 +272,16 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
   }
   return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                              qkv_dtype, o, hT, stream);
+}
+
+int kda_chunk_fwd_static(const void* q, const void* k, const void* v, const float* log_alpha,
+                         const float* beta, const float* h0, const int32_t* cu_seqlens,
+                         int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                         void* o, float* hT, cudaStream_t stream) {
+  void* scratch = nullptr;
+  if (cudaGetSymbolAddress(&scratch, g_kda_static_scratch) != cudaSuccess) return KDA_ERR_CUDA;
+  return kda_chunk_fwd_ws(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                          qkv_dtype, o, hT, scratch, STATIC_SCRATCH_BYTES, stream);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,

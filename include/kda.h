@@ -131,6 +131,21 @@ size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_h
                                     kda_dtype qkv_dtype, int has_cu_seqlens);
 
 /*
+ * kda_chunk_fwd_static - kda_chunk_fwd_ws with the library's own scratch: a 16 MiB
+ * device array that is part of the loaded module (set up with
+ * cudaGetSymbolAddress), so the call allocates nothing and needs no workspace
+ * argument. Same arguments, results and errors as kda_chunk_fwd; the time split
+ * runs whenever its workspace fits the array. Calls through this entry point share
+ * the one array: they must not overlap in time (issue them on one stream, or order
+ * them), and a call must not overlap a kda_chunk_fwd_static call on another device
+ * context using the same module.
+ */
+int kda_chunk_fwd_static(const void* q, const void* k, const void* v, const float* log_alpha,
+                         const float* beta, const float* h0, const int32_t* cu_seqlens,
+                         int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                         void* o, float* hT, cudaStream_t stream);
+
+/*
  * kda_chunk_fwd_simt - the same operation as kda_chunk_fwd, always on the fp32
  * CUDA-core chunk kernel (exact element-wise decay factors, fp32 math). Same
  * arguments, layouts and errors. It is the precision path for fp32 inputs and a

@@ -41,6 +41,37 @@ DECODE_BYTES_PER_CHAIN = 2 * STATE_BYTES + 4 * 2 * D + 2 + 2 * D   # state rw + 
 L2_BYTES = 126 * 1024 * 1024
 
 
+def _source_hash() -> str:
+    """sha256 prefix of the kernel sources (csrc/*.cu, csrc/*.cuh, include/kda.h)."""
+    import glob
+    import hashlib
+    csrc = os.path.join(ROOT, "channel_wise_gated_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")))
+    files.append(os.path.join(ROOT, "include", "kda.h"))
+    h = hashlib.sha256()
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(split: bool, token_heads: int):
+    """DRAM bytes per prefill call from the committed ncu summary, scaled to this
+    workload by its token-heads, or None when the kernel sources changed since the
+    capture (or the capture does not describe this kind of call)."""
+    import re
+    path = os.path.join(ROOT, "profiles", "kda_chunk_tc_prefill4k_full.md")
+    if not split or not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    mh = re.search(r"^source_hash: ([0-9a-f]+)$", txt, re.M)
+    mb = re.search(r"^split_call_dram_bytes_per_token_head: ([0-9.]+)$", txt, re.M)
+    if not mh or not mb or mh.group(1) != _source_hash():
+        return None
+    return float(mb.group(1)) * token_heads
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -411,7 +442,11 @@ def main():
                        "l2": f"inputs larger than L2 ({step_bytes / 1e9:.1f} GB per step)",
                        "parallelism": f"replicas x{ws}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved / hbm_peak, "traffic": None,
+                         "frac": achieved / hbm_peak,
+                         "traffic": _profiled_traffic(split, T * H),
+                         "traffic_note": ("DRAM bytes per call from the ncu capture of "
+                                          "profiles/kda_chunk_tc_prefill4k_full.md, scaled by "
+                                          "token-heads; null if the kernel changed since"),
                          "peak_kind": peak_kind,
                          "kernel": "kda_chunk_tc_kernel",
                          "unit_of_work": ("one prefill call (state pass + segment scan + "

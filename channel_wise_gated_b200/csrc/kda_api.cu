@@ -132,10 +132,23 @@ size_t segment_workspace_bytes(int n_seg, int32_t n_heads) {
   return n_seg >= 3 ? (size_t)kda::seg::slots(n_seg) * n_heads * kda::D * kda::D * sizeof(float) : 0;
 }
 
+// Packed batches: a launch order by decreasing length (one int32 per sequence),
+// worth it once the CTAs exceed one wave; ranking is O(n^2) so it stays bounded.
+constexpr int32_t MAX_ORDERED_SEQS = 16384;
+size_t order_workspace_bytes(int32_t n_seqs, int32_t n_heads) {
+  if (n_seqs < 2 || n_seqs > MAX_ORDERED_SEQS) return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  if ((int64_t)n_seqs * n_heads <= sms) return 0;
+  return ((size_t)n_seqs * sizeof(int32_t) + 255) & ~(size_t)255;
+}
+
 int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
                     const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                     int64_t t_total, int32_t n_heads, void* o, float* hT, int n_seg,
-                    float* seg_states, cudaStream_t stream) {
+                    float* seg_states, int32_t* seq_order, cudaStream_t stream) {
   using namespace kda::tc;
   const uint64_t cols = (uint64_t)n_heads * kda::D;
   const uint64_t rows = (uint64_t)t_total;
@@ -168,6 +181,14 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.n_seg = 0;
   a.seg_chunks = 0;
   a.seg_states = nullptr;
+  a.seq_order = nullptr;
+  if (seq_order != nullptr && cu_seqlens != nullptr && n_seqs > 1) {
+    const unsigned blocks = (unsigned)((n_seqs + kda::seg::ORDER_THREADS - 1) / kda::seg::ORDER_THREADS);
+    kda::seg::kda_seq_order_kernel<<<blocks, kda::seg::ORDER_THREADS, 0, stream>>>(
+        cu_seqlens, n_seqs, t_total, seq_order);
+    if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
+    a.seq_order = seq_order;
+  }
   if (n_seg < 3 || seg_states == nullptr) {
     const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
     kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
@@ -253,7 +274,11 @@ size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_h
   static const int32_t dummy = 0;
   const int n_seg = plan_segments(has_cu_seqlens ? &dummy : nullptr, n_seqs, t_total, n_heads,
                                   qkv_dtype);
-  return segment_workspace_bytes(n_seg, n_heads);
+  if (n_seg >= 3) return segment_workspace_bytes(n_seg, n_heads);
+  if (has_cu_seqlens && n_seqs > 1 &&
+      use_tc(&dummy, n_seqs, t_total, n_heads, qkv_dtype))
+    return order_workspace_bytes(n_seqs, n_heads);
+  return 0;
 }
 
 int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* log_alpha,
@@ -267,8 +292,12 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
   if (use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype)) {
     int n_seg = plan_segments(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype);
     if (workspace == nullptr || workspace_bytes < segment_workspace_bytes(n_seg, n_heads)) n_seg = 0;
+    int32_t* order = nullptr;
+    const size_t ob = order_workspace_bytes(n_seqs, n_heads);
+    if (n_seg == 0 && cu_seqlens != nullptr && workspace != nullptr && ob > 0 && workspace_bytes >= ob)
+      order = static_cast<int32_t*>(workspace);
     return launch_chunk_tc(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads, o,
-                           hT, n_seg, static_cast<float*>(workspace), stream);
+                           hT, n_seg, static_cast<float*>(workspace), order, stream);
   }
   return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                              qkv_dtype, o, hT, stream);

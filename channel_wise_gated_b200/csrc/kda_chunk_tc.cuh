@@ -166,6 +166,7 @@ struct Args {
   int n_seg;
   int seg_chunks;
   float* seg_states;   // [3 n_seg - 5][H][128][128]
+  const int32_t* seq_order;   // PLAN_SEQ: sequences longest first (or null: index order)
 };
 
 struct Ctx {
@@ -1196,8 +1197,15 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.write_o = true;
   const size_t state_elems = (size_t)D * D;
   if (args.plan == PLAN_SEQ) {
-    seq_bounds(args.cu_seqlens, slot, args.n_seqs, args.t_total, x.bos, x.eos);
-    const size_t sidx = ((size_t)slot * H + x.h) * state_elems;
+    // CTAs start in index order; with seq_order the longest sequences go first, so
+    // the last wave holds short ones
+    int n = slot;
+    if (args.seq_order) {
+      const int o = args.seq_order[slot];
+      n = (o >= 0 && o < args.n_seqs) ? o : slot;
+    }
+    seq_bounds(args.cu_seqlens, n, args.n_seqs, args.t_total, x.bos, x.eos);
+    const size_t sidx = ((size_t)n * H + x.h) * state_elems;
     x.h0 = args.h0 ? args.h0 + sidx : nullptr;
     x.hT = args.hT ? args.hT + sidx : nullptr;
   } else {

@@ -74,5 +74,39 @@ kda_segment_scan_kernel(float* __restrict__ states, int n_heads, int n_seg) {
   }
 }
 
+// Launch order of a packed batch: order[rank] = sequence, ranked by decreasing
+// length (ties by index), so that the chunk kernel starts the longest sequences
+// first. Thread i ranks sequence i against all others; lengths are clamped like
+// the chunk kernel clamps them (a bad cu_seqlens only changes the order).
+constexpr int ORDER_THREADS = 256;
+constexpr int ORDER_TILE = 1024;
+
+__global__ void __launch_bounds__(ORDER_THREADS)
+kda_seq_order_kernel(const int32_t* __restrict__ cu, int n_seqs, int64_t t_total,
+                     int32_t* __restrict__ order) {
+  __shared__ int64_t len_tile[ORDER_TILE];
+  const int i = blockIdx.x * ORDER_THREADS + threadIdx.x;
+  auto len_of = [&](int s) -> int64_t {
+    const int64_t a = cu[s], b = cu[s + 1];
+    const int64_t ca = a < 0 ? 0 : (a > t_total ? t_total : a);
+    const int64_t cb = b < ca ? ca : (b > t_total ? t_total : b);
+    return cb - ca;
+  };
+  const int64_t li = i < n_seqs ? len_of(i) : 0;
+  int rank = 0;
+  for (int t0 = 0; t0 < n_seqs; t0 += ORDER_TILE) {
+    const int tn = (n_seqs - t0) < ORDER_TILE ? (n_seqs - t0) : ORDER_TILE;
+    __syncthreads();
+    for (int k = threadIdx.x; k < tn; k += ORDER_THREADS) len_tile[k] = len_of(t0 + k);
+    __syncthreads();
+    if (i < n_seqs)
+      for (int k = 0; k < tn; ++k) {
+        const int64_t lj = len_tile[k];
+        rank += (lj > li || (lj == li && t0 + k < i)) ? 1 : 0;
+      }
+  }
+  if (i < n_seqs) order[rank] = i;
+}
+
 }  // namespace seg
 }  // namespace kda

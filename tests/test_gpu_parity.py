@@ -229,6 +229,24 @@ def test_time_split_16_heads_mixed_decay(kda):
     assert rel_err(hT, h_ref) <= TOL_BF16
 
 
+def test_packed_batch_longest_first(kda):
+    """A packed batch with more CTAs than SMs is launched longest sequence first (the
+    order lives in the workspace): same results as index order, and the oracle's."""
+    lens = [64 * 3 + 5, 0, 900, 64, 1, 2000, 64 * 20, 333, 0, 1500] * 4
+    H = 16
+    assert len(lens) * H > 148
+    inp = kda_inputs.make_prefill(lens, H, torch.bfloat16, torch.float32, 3.0, True, seed=85,
+                                  device="cuda")
+    lib = kda._native.load()
+    assert lib.kda_chunk_fwd_workspace_size(len(lens), sum(lens), H, kda._native.KDA_BF16, 1) > 0
+    o_a, h_a = _run(kda, inp, kernel="auto")      # ordered (workspace)
+    o_s, h_s = _run(kda, inp, kernel="single")    # index order (no workspace)
+    assert torch.equal(o_a, o_s) and torch.equal(h_a, h_s)
+    o_ref, h_ref = _oracle(inp)
+    assert rel_err(o_a, o_ref) <= TOL_BF16
+    assert rel_err(h_a, h_ref) <= TOL_BF16
+
+
 def test_time_split_equals_single_pass(kda):
     """The split and the single pass compute the same recurrence."""
     T, H = 64 * 64, 32

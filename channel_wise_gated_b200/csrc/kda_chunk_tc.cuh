@@ -41,9 +41,10 @@
 //   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars;
 //               its first thread issues the k/q TMA loads and the L2 prefetch of the
 //               log-decay
-//   warps 8-11  prep B (chunk c+1): Gram readout, UT solve, T*beta tile, W' tile;
-//               its first thread issues the Gram and W' products
-//   warps 12-19 state  (chunk c):   decay S in TMEM and write S'', Delta tile, output;
+//   warps 8-11  prep B (chunk c+1): Gram readout, UT solve, T*beta tile; its first
+//               thread issues the Gram and W' products
+//   warps 12-19 state  (chunk c):   decay S in TMEM and write S'', the -W' tile, Delta
+//               tile, output;
 //               its first thread issues the state products, U and the v TMA loads
 // Every mbarrier wait is bounded; a timeout flags KDA_ERR_TIMEOUT and every role
 // leaves (a group keeps meeting at its own named barriers, doing no work).
@@ -126,12 +127,12 @@ enum : int {
   B_TB = 10,        // P and T*beta tiles written
   B_WDONE = 11,     // W' MMA done
   B_UDONE = 12,     // U MMA done (v and T*beta free)
-  B_READY = 13,     // [2] -W' tile written
+  B_WREAD = 13,     // -W' read out of TMEM (by the state warps)
   B_CRIT = 15,      // [O | Delta] product done
   B_ZDONE = 16,     // state update product done
   B_PD = 17,        // P Delta product done (output complete)
   B_CKFREE = 18,    // [2] Ck/P slot no longer needed
-  B_WFREE = 20,     // prep B done with a chunk (-W' read out, workspace free)
+  B_WFREE = 20,     // prep B done with a chunk (workspace free)
   B_FIN_C = 21,     // drains
   B_FIN_P = 22,
   NUM_BARS = 23
@@ -782,8 +783,9 @@ __device__ void prep_b_role(const Ctx& x) {
       }
       tc_fence_before();
     }
-    // the previous chunk's U product must be done reading the T*beta tile
-    ok = ok && ((c < 1) || wait_b(x, B_UDONE, (c - 1) & 1));
+    // the previous chunk's U and W' products must be done reading the T*beta tile (U
+    // may go out before W' completes, from another thread: its commit does not cover W')
+    ok = ok && ((c < 1) || (wait_b(x, B_UDONE, (c - 1) & 1) && wait_b(x, B_WDONE, (c - 1) & 1)));
     if (named_bar_or(BAR_PB, PB_THREADS, !ok)) break;
     // the Gram columns are free again: the next chunk's Gram goes out now if its
     // tiles are already written
@@ -913,36 +915,10 @@ __device__ void prep_b_role(const Ctx& x) {
     named_bar_sync(BAR_PB, PB_THREADS);
     if (tid == 0) {
       mbar_arrive(&x.bars[B_TB]);
-      issue_w(x, c);
-    }
-
-    // ---- -W' readout: lane = channel ch, columns = rows r; one 2-byte store per row
-    //      (a warp covers 64 contiguous bytes of a row)
-    ok = wait_b(x, B_WDONE, c & 1);
-    tc_fence_after();
-    {
-      const int ch = 32 * q + lane;
-      uint8_t* wt = kq + koff + (ch >> 6) * 16384;
-      const uint32_t cb = (uint32_t)(ch & 63) * 2u;
-#pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        float v[32];
-        tmem_ld32(x.tmem + TM_W + lane_base + 32 * half, v);
-        tmem_ld_wait();
-        if (ok) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            *reinterpret_cast<__nv_bfloat16*>(wt + swz128((32 * half + i) * 128 + cb)) =
-                __float2bfloat16_rn(v[i]);
-        }
-      }
-    }
-    tc_fence_before();
-    fence_proxy_async_smem();
-    if (named_bar_or(BAR_PB, PB_THREADS, !ok)) break;
-    if (tid == 0) {
-      mbar_arrive(&x.bars[B_READY + (c & 1)]);
-      mbar_arrive(&x.bars[B_WFREE]);
+      // W' of this chunk once the state warps have read out the previous one (they
+      // read it out themselves, right before their [O | Delta] product)
+      if (c == 0 || wait_b(x, B_WREAD, (c - 1) & 1)) issue_w(x, c);
+      mbar_arrive(&x.bars[B_WFREE]);   // done with this chunk: the workspace is free
     }
   }
   if (tid == 0) drain(x, B_FIN_P);
@@ -1067,6 +1043,25 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     return true;
   };
 
+  // -W' of chunk cc (TMEM, lane j = key channel, columns = rows) -> the k half of the
+  // chunk's stage tile, rows 32hh..32hh+31: the B operand of the [O | Delta] product
+  auto w_readout = [&](int cc) -> bool {
+    if (!wait_b(x, B_WDONE, cc & 1)) return false;
+    tc_fence_after();
+    uint8_t* wt = x.sm + OFF_KQ + (cc % 3) * KQ_BYTES + ((cc & 1) ? 8192 : 0) + (j >> 6) * 16384;
+    const uint32_t cb = (uint32_t)(j & 63) * 2u;
+    float v[32];
+    tmem_ld32(x.tmem + TM_W + lb + 32 * hh, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      *reinterpret_cast<__nv_bfloat16*>(wt + swz128((32 * hh + i) * 128 + cb)) =
+          __float2bfloat16_rn(v[i]);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    return true;
+  };
+
   bool alive = true;
   if (n > 0) {
     if (issuer) {
@@ -1075,9 +1070,11 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     }
     alive = wait_b(x, B_TILES + 0, 0);
     if (alive) s_pass(0);
+    alive = alive && w_readout(0);
     named_bar_sync(BAR_ST, ST_THREADS);
     if (issuer && alive) {
-      alive = issue_u_of(0, true) && wait_b(x, B_READY + 0, 0);
+      mbar_arrive(&x.bars[B_WREAD]);
+      alive = issue_u_of(0, true);
       if (alive) issue_crit(x, 0);
     }
   }
@@ -1119,10 +1116,11 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         tc_fence_after();
         s_pass(c + 1);
       }
+      alive = alive && w_readout(c + 1);
       named_bar_sync(BAR_ST, ST_THREADS);
       if (issuer && alive) {
+        mbar_arrive(&x.bars[B_WREAD]);
         if (u_issued < c + 2) alive = issue_u_of(c + 1, true);
-        alive = alive && wait_b(x, B_READY + ((c + 1) & 1), ((c + 1) >> 1) & 1);
         if (alive) issue_crit(x, c + 1);
       }
     }

@@ -734,10 +734,8 @@ __device__ void prep_b_role(const Ctx& x) {
 
   for (int c = 0; c < x.n_chunks; ++c) {
     const int s3 = c % 3;
-    uint8_t* kq = x.sm + OFF_KQ + s3 * KQ_BYTES;
     uint8_t* ck = x.sm + OFF_CKP + (c & 1) * CKP_BYTES;
     const float* betas = reinterpret_cast<const float*>(x.sm + OFF_BETA) + s3 * 64;
-    const uint32_t koff = (c & 1) ? 8192u : 0u;
 
     bool ok = wait_b(x, B_TILES + (c & 1), (c >> 1) & 1);
     const bool exact = ok && xflag[s3] != 0;

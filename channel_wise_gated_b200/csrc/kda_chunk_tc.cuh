@@ -38,11 +38,10 @@
 // c+1 is already accumulating.
 //
 // Roles (640 threads), a pipeline three chunks deep:
-//   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars;
-//               its first thread issues the k/q TMA loads and the L2 prefetch of the
-//               log-decay
+//   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars
 //   warps 8-11  prep B (chunk c+1): Gram readout, UT solve, T*beta tile; its first
-//               thread issues the Gram and W' products
+//               thread issues the Gram and W' products, the k/q TMA loads and the L2
+//               prefetch of the log-decay
 //   warps 12-19 state  (chunk c):   decay S in TMEM and write S'', the -W' tile, Delta
 //               tile, output;
 //               its first thread issues the state products, U and the v TMA loads
@@ -492,8 +491,7 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, i
   return true;
 }
 
-__device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_k,
-                            const CUtensorMap* map_q, const CUtensorMap* map_la) {
+__device__ void prep_a_role(const Ctx& x, const Args& p) {
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
   const int kb = lane >> 4;                // kblock of this thread's 4 channels
@@ -502,30 +500,13 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
   float* wsum = reinterpret_cast<float*>(x.sm + OFF_WSUM);
   float* grow = reinterpret_cast<float*>(x.sm + OFF_GROW);
   int* xflag = reinterpret_cast<int*>(x.sm + OFF_XFLAG);
-  const int xk = x.h * D;
-  // (thread 0) k/q loads go out as soon as their stage slot is free (its previous
-  // chunk's state product done), up to two chunks ahead of this role; the
-  // log-decay is prefetched into L2 three chunks ahead. Never blocks unless this
-  // role would otherwise wait for the tiles itself.
-  int kq_issued = 0, kq_landed = 0;
-  auto push_kq = [&](int upto, bool block) {
-    while (kq_issued < x.n_chunks && kq_issued <= upto) {
-      const int cn = kq_issued;
-      if (cn >= 3) {
-        uint64_t* fb = &x.bars[B_KQFREE + cn % 3];
-        const uint32_t par = ((cn - 3) / 3) & 1;
-        if (block ? !wait_b(x, B_KQFREE + cn % 3, par) : !mbar_test_wait(fb, par)) return;
-      }
-      issue_kq(x, map_k, map_q, cn);
-      if (cn + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
-      ++kq_issued;
-    }
+  // beta of row tid of chunk cn (zero past the end of the sequence), loaded one chunk
+  // early so that its latency hides behind a whole chunk of work
+  auto load_beta = [&](int cn) -> float {
+    const int64_t t = x.bos + (int64_t)cn * CHUNK + tid;
+    return (tid < 64 && t < x.eos) ? ldg_nc_f32(p.beta + (size_t)t * p.n_heads + x.h) : 0.f;
   };
-  if (tid == 0) {
-    for (int c = 0; c < 3 && c < x.n_chunks; ++c)
-      tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)c * CHUNK));
-    push_kq(1, false);
-  }
+  float beta_next = load_beta(0);
 
   for (int c = 0; c < x.n_chunks; ++c) {
     const int s3 = c % 3;
@@ -537,8 +518,8 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
     float* betas = reinterpret_cast<float*>(x.sm + OFF_BETA) + s3 * 64;
     float* scal = reinterpret_cast<float*>(x.sm + OFF_SCAL) + s3 * 256;
 
-    // log-decay rows 8w..8w+7 of this chunk, channels c0..c0+3 (L2-prefetched by the
-    // TMA thread three chunks ahead); zero past the end of the sequence
+    // log-decay rows 8w..8w+7 of this chunk, channels c0..c0+3 (L2-prefetched three
+    // chunks ahead by the thread that loads k/q); zero past the end of the sequence
     float g2[8][4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -549,13 +530,8 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
     }
     // (the reader of this beta slot, prep B three chunks back, finished before this
     // role got the Ck slot of chunk c-1)
-    if (tid < 64)
-      betas[tid] = (t0 + tid < x.eos) ? ldg_nc_f32(p.beta + (size_t)(t0 + tid) * p.n_heads + x.h) : 0.f;
-    // loads in flight: thread 0 tops up the k/q loads (this chunk's must be out)
-    if (tid == 0) {
-      push_kq(c, true);
-      push_kq(c + 2, false);
-    }
+    if (tid < 64) betas[tid] = beta_next;
+    beta_next = load_beta(c + 1);
 
     // ---- inclusive cumsum over rows, in log2 units
     {
@@ -584,7 +560,6 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
       if (w == 7) *reinterpret_cast<float4*>(&grow[128 + c0]) = make_float4(g2[7][0], g2[7][1], g2[7][2], g2[7][3]);
     }
     bool ok = wait_b(x, B_FULL + s3, (c / 3) & 1);
-    if (ok) kq_landed = c + 1;
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
 
     // ---- range guard: max over channels of G_0 - G_63
@@ -638,14 +613,8 @@ __device__ void prep_a_role(const Ctx& x, const Args& p, const CUtensorMap* map_
     }
     fence_proxy_async_smem();
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
-    if (tid == 0) {
-      mbar_arrive(&x.bars[B_TILES + (c & 1)]);
-      push_kq(c + 2, false);
-    }
+    if (tid == 0) mbar_arrive(&x.bars[B_TILES + (c & 1)]);
   }
-  // never leave with copies in flight
-  if (tid == 0)
-    for (int c = kq_landed; c < kq_issued; ++c) settle(&x.bars[B_FULL + c % 3], (c / 3) & 1);
 }
 
 // ============================================================================
@@ -718,7 +687,8 @@ __device__ __forceinline__ void issue_gram(const Ctx& x, int g) {
   umma_commit(&x.bars[B_GRAM]);
 }
 
-__device__ void prep_b_role(const Ctx& x) {
+__device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
+                            const CUtensorMap* map_la) {
   const int tid = threadIdx.x - PB_WARP0 * 32;
   const int q = tid >> 5, lane = tid & 31;   // q = warp within the group = TMEM lane quarter
   const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -728,6 +698,30 @@ __device__ void prep_b_role(const Ctx& x) {
   auto A = [&](int a, int b) { return aw + (16 * a) * AW + 16 * b; };
   uint8_t* tt = x.sm + OFF_TB;
   int gram_issued = 0;   // (thread 0) Gram products issued so far
+  // (thread 0) the k/q loads of the CTA: each goes out once its stage slot is free
+  // (the [O | Delta] product of the chunk three back done), and prefetches the
+  // log-decay of the chunk three later into L2. Polled at a few points of every
+  // chunk; chunk c+1's is waited for at the start of chunk c (prep A needs it next).
+  const int xk = x.h * D;
+  int kq_issued = 0;
+  auto push_kq = [&](int upto, bool block) {
+    while (kq_issued < x.n_chunks && kq_issued <= upto) {
+      const int cn = kq_issued;
+      if (cn >= 3) {
+        uint64_t* fb = &x.bars[B_KQFREE + cn % 3];
+        const uint32_t par = ((cn - 3) / 3) & 1;
+        if (block ? !wait_b(x, B_KQFREE + cn % 3, par) : !mbar_test_wait(fb, par)) return;
+      }
+      issue_kq(x, map_k, map_q, cn);
+      if (cn + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
+      ++kq_issued;
+    }
+  };
+  if (tid == 0) {
+    for (int c = 0; c < 3 && c < x.n_chunks; ++c)
+      tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)c * CHUNK));
+    push_kq(2, false);
+  }
   // blocks above the diagonal of the T*beta tile stay zero for the whole kernel
   for (int i = tid; i < 512; i += PB_THREADS)
     *reinterpret_cast<uint4*>(tt + i * 16) = make_uint4(0u, 0u, 0u, 0u);
@@ -737,6 +731,10 @@ __device__ void prep_b_role(const Ctx& x) {
     uint8_t* ck = x.sm + OFF_CKP + (c & 1) * CKP_BYTES;
     const float* betas = reinterpret_cast<const float*>(x.sm + OFF_BETA) + s3 * 64;
 
+    if (tid == 0) {
+      push_kq(c + 1, true);
+      push_kq(c + 2, false);
+    }
     bool ok = wait_b(x, B_TILES + (c & 1), (c >> 1) & 1);
     const bool exact = ok && xflag[s3] != 0;
     // the Gram of this chunk, unless it went out while the previous chunk was solved
@@ -781,6 +779,7 @@ __device__ void prep_b_role(const Ctx& x) {
       }
       tc_fence_before();
     }
+    if (tid == 0) push_kq(c + 2, false);
     // the previous chunk's U and W' products must be done reading the T*beta tile (U
     // may go out before W' completes, from another thread: its commit does not cover W')
     ok = ok && ((c < 1) || (wait_b(x, B_UDONE, (c - 1) & 1) && wait_b(x, B_WDONE, (c - 1) & 1)));
@@ -917,9 +916,16 @@ __device__ void prep_b_role(const Ctx& x) {
       // read it out themselves, right before their [O | Delta] product)
       if (c == 0 || wait_b(x, B_WREAD, (c - 1) & 1)) issue_w(x, c);
       mbar_arrive(&x.bars[B_WFREE]);   // done with this chunk: the workspace is free
+      push_kq(c + 2, false);
     }
   }
-  if (tid == 0) drain(x, B_FIN_P);
+  if (tid == 0) {
+    drain(x, B_FIN_P);
+    // never leave with copies in flight: the last load into each slot has landed (an
+    // earlier one into the same slot was consumed before that load went out)
+    for (int cn = (kq_issued > 3 ? kq_issued - 3 : 0); cn < kq_issued; ++cn)
+      settle(&x.bars[B_FULL + cn % 3], (cn / 3) & 1);
+  }
 }
 
 // ---- cold paths of the state warps, out of line with scalar arguments (they run
@@ -1258,9 +1264,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.tmem = *tmem_slot;
 
   if (warp < PA_WARPS) {
-    prep_a_role(x, args, &map_k, &map_q, &map_la);
+    prep_a_role(x, args);
   } else if (warp < ST_WARP0) {
-    prep_b_role(x);
+    prep_b_role(x, &map_k, &map_q, &map_la);
   } else {
     state_role(x, args, &map_v, &map_o);
   }

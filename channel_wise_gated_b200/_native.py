@@ -24,6 +24,7 @@ KDA_ERR_ALIGN = -4
 KDA_ERR_SEQLENS = -5
 KDA_ERR_CUDA = -6
 KDA_ERR_TIMEOUT = -7
+KDA_ERR_SCRATCH = -8
 
 # entry point -> argument types (all return int except kda_status_string)
 _P, _I32, _I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64

@@ -15,11 +15,11 @@
 #include "kda_decode.cuh"
 #include "kda_segment.cuh"
 
-// Scratch of kda_chunk_fwd_static: module-resident device memory (no allocation at
-// call time), large enough for the time split of any head count on a 148-SM part
-// (slots x heads <= 3 x 74 + 5, 64 KiB each).
-constexpr size_t STATIC_SCRATCH_BYTES = (size_t)16 << 20;
-static __device__ __align__(256) unsigned char g_kda_static_scratch[STATIC_SCRATCH_BYTES];
+// Scratch of kda_chunk_fwd_static, for callers that cannot allocate device memory:
+// a fixed array in every GPU context that loads the library. It covers the time
+// split of any head count on a 148-SM part (at most 220 slots x 64 KiB = 13.75 MiB);
+// larger needs are rejected with KDA_ERR_SCRATCH.
+static __device__ __align__(256) unsigned char g_kda_static_scratch[KDA_STATIC_SCRATCH_BYTES];
 
 namespace {
 
@@ -245,6 +245,28 @@ int launch_decode(const void* q, const void* k, const void* v, const void* log_a
   return launch_status();
 }
 
+// Device address of g_kda_static_scratch on the current device. In host code the
+// array's name only stands in for the symbol, so the address is looked up once per
+// device, with that device current, and kept.
+constexpr int MAX_STATIC_DEVICES = 64;
+std::mutex g_static_mu;
+void* g_static_addr[MAX_STATIC_DEVICES] = {};
+
+int static_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_STATIC_DEVICES)
+    return KDA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (g_static_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kda_static_scratch) != cudaSuccess || p == nullptr)
+      return KDA_ERR_CUDA;
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return KDA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -307,10 +329,17 @@ int kda_chunk_fwd_static(const void* q, const void* k, const void* v, const floa
                          const float* beta, const float* h0, const int32_t* cu_seqlens,
                          int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
                          void* o, float* hT, cudaStream_t stream) {
+  const int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
+                                     n_heads, qkv_dtype, o, hT);
+  if (st != KDA_OK) return st;
+  if (kda_chunk_fwd_workspace_size(n_seqs, t_total, n_heads, qkv_dtype, cu_seqlens != nullptr) >
+      KDA_STATIC_SCRATCH_BYTES)
+    return KDA_ERR_SCRATCH;
   void* scratch = nullptr;
-  if (cudaGetSymbolAddress(&scratch, g_kda_static_scratch) != cudaSuccess) return KDA_ERR_CUDA;
+  const int sst = static_scratch_address(&scratch);
+  if (sst != KDA_OK) return sst;
   return kda_chunk_fwd_ws(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
-                          qkv_dtype, o, hT, scratch, STATIC_SCRATCH_BYTES, stream);
+                          qkv_dtype, o, hT, scratch, KDA_STATIC_SCRATCH_BYTES, stream);
 }
 
 int kda_decode_step(const void* q, const void* k, const void* v, const void* log_alpha,
@@ -366,6 +395,8 @@ const char* kda_status_string(int status) {
     case KDA_ERR_SEQLENS: return "KDA_ERR_SEQLENS: cu_seqlens inconsistent";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA call or launch failed";
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    case KDA_ERR_SCRATCH:
+      return "KDA_ERR_SCRATCH: the call needs more scratch than the library's static array holds";
     default: return "unknown kda_status";
   }
 }

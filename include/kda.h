@@ -28,7 +28,8 @@
  *   - Head dimension is fixed: d_k = d_v = 128.
  *   - Every pointer is a DEVICE pointer owned by the caller. The library
  *     allocates no device memory and keeps no per-call state (scratch, where an
- *     entry point can use it, is a caller-provided workspace).
+ *     entry point can use it, is a caller-provided workspace, or for
+ *     kda_chunk_fwd_static a fixed array compiled into the library).
  *   - Calls are asynchronous and ordered on `stream`. A return of KDA_OK means
  *     "arguments validated and kernel launched"; device-side problems (bad
  *     cu_seqlens contents) are reported later by kda_device_status().
@@ -57,7 +58,9 @@ typedef enum {
   KDA_ERR_ALIGN = -4,    /* a tensor pointer is not 16-byte aligned */
   KDA_ERR_SEQLENS = -5,  /* cu_seqlens inconsistent (host check, or reported by the device) */
   KDA_ERR_CUDA = -6,     /* a CUDA runtime call or kernel launch failed */
-  KDA_ERR_TIMEOUT = -7   /* a kernel gave up a bounded wait and skipped its work */
+  KDA_ERR_TIMEOUT = -7,  /* a kernel gave up a bounded wait and skipped its work */
+  KDA_ERR_SCRATCH = -8   /* kda_chunk_fwd_static: the call needs more scratch than
+                            KDA_STATIC_SCRATCH_BYTES; nothing was launched */
 } kda_status;
 
 /*
@@ -131,15 +134,42 @@ size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_h
                                     kda_dtype qkv_dtype, int has_cu_seqlens);
 
 /*
- * kda_chunk_fwd_static - kda_chunk_fwd_ws with the library's own scratch: a 16 MiB
- * device array that is part of the loaded module (set up with
- * cudaGetSymbolAddress), so the call allocates nothing and needs no workspace
- * argument. Same arguments, results and errors as kda_chunk_fwd; the time split
- * runs whenever its workspace fits the array. Calls through this entry point share
- * the one array: they must not overlap in time (issue them on one stream, or order
- * them), and a call must not overlap a kda_chunk_fwd_static call on another device
- * context using the same module.
+ * kda_chunk_fwd_static - kda_chunk_fwd for callers that cannot allocate device
+ * memory. The Kimi Linear pages have no counterpart to this entry point: it is a
+ * deployment variant of kda_chunk_fwd_ws whose scratch is a fixed array compiled
+ * into this library instead of a buffer from the caller.
+ *
+ * Who cannot allocate: an op that runs as a plugin or custom kernel inside an
+ * inference engine which has already reserved the GPU's memory for its own pool
+ * and hands the op only its inputs and outputs (a cudaMalloc there fails, or eats
+ * into memory the engine has promised elsewhere), and code on a latency-critical
+ * path, where cudaMalloc and cudaFree are ruled out because they can synchronise
+ * the whole device. Such callers still pass q, k, v, the gates, o and hT.
+ *
+ * Scratch: one __device__ array of KDA_STATIC_SCRATCH_BYTES (16 MiB), 256-byte
+ * aligned, in every GPU context that loads the library, held until the process
+ * exits. The time split of one long sequence uses (3n - 5) * n_heads * 64 KiB of
+ * it (n segments; at most 13.75 MiB on a 148-SM B200) and a packed batch of more
+ * CTAs than SMs uses 4 bytes per sequence.
+ *
+ * Limit: a call for which kda_chunk_fwd_workspace_size(...) exceeds
+ * KDA_STATIC_SCRATCH_BYTES is rejected with KDA_ERR_SCRATCH before anything is
+ * launched (on a 148-SM B200 no call reaches it; parts with more SMs can).
+ *
+ * Set-up: the first call on each device, made with that device current, looks up
+ * the array's device address (cudaGetSymbolAddress, which may load this library's
+ * kernels onto the device) and keeps it for later calls; make that first call
+ * before any stream capture on the device. A failed look-up returns KDA_ERR_CUDA.
+ *
+ * Sharing: every call on a device, from any stream or host thread, uses the same
+ * array and leaves its contents behind. Nothing in it has to start at zero (each
+ * call writes every scratch byte it reads before reading it), but calls whose
+ * kernels overlap on the GPU race on the array and give wrong results: issue them
+ * on one stream, or order them with events.
+ *
+ * Arguments, layouts, results and other errors: as kda_chunk_fwd.
  */
+#define KDA_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
 int kda_chunk_fwd_static(const void* q, const void* k, const void* v, const float* log_alpha,
                          const float* beta, const float* h0, const int32_t* cu_seqlens,
                          int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,

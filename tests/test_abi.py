@@ -42,9 +42,10 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for st in range(0, -8, -1):
+    for st in range(0, -9, -1):
         s = _native.status_string(st)
         assert s.startswith("KDA_")
+    assert "scratch" in _native.status_string(_native.KDA_ERR_SCRATCH)
     assert "unknown" in _native.status_string(-99)
 
 
@@ -78,6 +79,14 @@ def test_chunk_validation(lib):
               FAKE, 1 << 20, None) == _native.KDA_ERR_NULL
     assert ws(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, _native.KDA_BF16, FAKE, None,
               FAKE + 8, 1 << 20, None) == _native.KDA_ERR_ALIGN
+    # the allocation-free entry point validates its arguments before it touches the device
+    st = lib.kda_chunk_fwd_static
+    assert st(None, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, _native.KDA_BF16, FAKE, None,
+              None) == _native.KDA_ERR_NULL
+    assert st(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 0, _native.KDA_BF16, FAKE, None,
+              None) == _native.KDA_ERR_SHAPE
+    assert st(FAKE, FAKE + 8, FAKE, FAKE, FAKE, None, None, 1, 64, 2, _native.KDA_BF16, FAKE,
+              None, None) == _native.KDA_ERR_ALIGN
 
 
 def test_workspace_size_queries(lib):

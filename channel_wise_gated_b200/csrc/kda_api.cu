@@ -164,7 +164,9 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
       !encode_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return KDA_ERR_CUDA;
-  if (cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(kda_chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)SMEM_BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(kda_chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess)
     return KDA_ERR_CUDA;
   Args a;
@@ -191,7 +193,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   }
   if (n_seg < 3 || seg_states == nullptr) {
     const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
-    kda_chunk_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
+    kda_chunk_tc_kernel<false><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
     return launch_status();
   }
   // time split: segment states, the scan over segments, then the outputs
@@ -200,7 +202,8 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.seg_chunks = (int)((n_chunks + n_seg - 1) / n_seg);
   a.seg_states = seg_states;
   a.plan = PLAN_STATES;
-  kda_chunk_tc_kernel<<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
+  // (the state pass writes no output: the lean instantiation)
+  kda_chunk_tc_kernel<true><<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
   if (n_seg > 2) {
@@ -213,7 +216,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
     if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
   }
   a.plan = PLAN_OUTPUTS;
-  kda_chunk_tc_kernel<<<(unsigned)(n_heads * n_seg), THREADS, SMEM_BYTES, stream>>>(
+  kda_chunk_tc_kernel<false><<<(unsigned)(n_heads * n_seg), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   return launch_status();
 }

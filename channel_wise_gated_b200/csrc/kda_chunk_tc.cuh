@@ -110,6 +110,7 @@ constexpr uint32_t TM_W = 448;    // -W'^T (M=128 channels, N=64 rows)
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_CRIT = idesc_bf16(128, 128, 0, 0);    // S''^T (TMEM) x stage tile
+constexpr uint32_t IDESC_DELTA = idesc_bf16(128, 64, 0, 0);    // S''^T (TMEM) x -W' (no output)
 constexpr uint32_t IDESC_Z = idesc_bf16(128, 128, 0, 1);       // Delta^T x Ck (MN-major)
 constexpr uint32_t IDESC_PD = idesc_bf16(128, 64, 0, 0);       // Delta^T x P
 constexpr uint32_t IDESC_GRAM = idesc_bf16(128, 64, 0, 0);     // stage tile x Ck
@@ -146,7 +147,10 @@ static_assert(NUM_BARS <= NBARS, "barrier slots");
 //     s = 1 .. n_seg-2      segment s from a zero state (R_s)
 //     s = n_seg-1 .. 2n-4   segment s-(n_seg-2) from the identity with v = 0 (its
 //                           transition M_s: S_end = M_s S_start + R_s)
-//   and each writes its final state to seg_states[s][h]; no output.
+//   and each writes its final state to seg_states[s][h]; no output. This pass runs
+//   the lean instantiation (LEAN = true): no q loads, no Rq tile, no P readout, the
+//   state product only for Delta (N=64), no P Delta product; with v = 0 also no U
+//   product (the Delta product starts from zero).
 //   PLAN_OUTPUTS (grid H x n_seg): segment j from its true entering state (the
 //     caller's h0, slot 0, or the scan's result in slot 2 n_seg - 5 + j), writing o,
 //     and the caller's hT for the last segment.
@@ -253,6 +257,7 @@ __device__ __forceinline__ uint64_t kdesc128(uint32_t addr) {
 // ============================================================================
 // TMA and MMA issue (each by the first thread of the role that consumes the result)
 // ============================================================================
+template <bool LEAN>
 __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* map_k,
                                          const CUtensorMap* map_q, int c) {
   const int xk = x.h * D;
@@ -260,9 +265,10 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* map_k,
   uint8_t* st = x.sm + OFF_KQ + (c % 3) * KQ_BYTES;
   const uint32_t koff = (c & 1) ? 8192u : 0u, qoff = 8192u - koff;
   uint64_t* full = &x.bars[B_FULL + c % 3];
-  mbar_arrive_expect_tx(full, 4 * 8192);
+  mbar_arrive_expect_tx(full, (LEAN ? 2 : 4) * 8192);
   tma_load_2d(st + koff, map_k, xk, y, full);
   tma_load_2d(st + 16384 + koff, map_k, xk + 64, y, full);
+  if (LEAN) return;   // no output: q is not needed
   tma_load_2d(st + qoff, map_q, xk, y, full);
   tma_load_2d(st + 16384 + qoff, map_q, xk + 64, y, full);
 }
@@ -291,19 +297,31 @@ __device__ void drain(const Ctx& x, int bar) {
 }
 
 // [O | Delta]^T (or [Delta | O]^T) += S''^T [stage tile]^T   (M=128, N=128, K=128);
-// the state operand comes from TMEM
+// the state operand comes from TMEM. Without output (LEAN) only Delta^T += S''^T (-W')^T
+// (N=64); with v = 0 there is no U to accumulate onto.
+template <bool LEAN>
 __device__ __forceinline__ void issue_crit(const Ctx& x, int c) {
   tc_fence_after();
   const uint32_t kq = smem_u32(x.sm) + OFF_KQ + (c % 3) * KQ_BYTES;
-  const uint32_t d = x.tmem + ((c & 1) ? TM_OA : TM_D);
+  if (LEAN) {
+    const uint32_t kh = kq + ((c & 1) ? 8192u : 0u);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    umma_bf16_tmem_a(d, x.tmem + TM_SB + kk * 8, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
-                     IDESC_CRIT, 1u);
+    for (int kk = 0; kk < 8; ++kk)
+      umma_bf16_tmem_a(x.tmem + TM_D, x.tmem + TM_SB + kk * 8,
+                       kdesc128(kh + (kk >> 2) * 16384 + (kk & 3) * 32), IDESC_DELTA,
+                       (kk == 0 && x.v_zero) ? 0u : 1u);
+  } else {
+    const uint32_t d = x.tmem + ((c & 1) ? TM_OA : TM_D);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      umma_bf16_tmem_a(d, x.tmem + TM_SB + kk * 8, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
+                       IDESC_CRIT, 1u);
+  }
   umma_commit(&x.bars[B_CRIT]);
   umma_commit(&x.bars[B_KQFREE + c % 3]);
 }
-// S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T
+// S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T (not without output)
+template <bool LEAN>
 __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   tc_fence_after();
   const uint32_t sbase = smem_u32(x.sm);
@@ -315,6 +333,10 @@ __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
     umma_bf16(x.tmem + TM_S, kdesc128(dt + kk * 32), make_sdesc(ck + kk * 2048, 8192, 1024, SWZ_128B),
               IDESC_Z, 1u);
   umma_commit(&x.bars[B_ZDONE]);
+  if (LEAN) {
+    umma_commit(&x.bars[B_CKFREE + (c & 1)]);
+    return;
+  }
   // (M=128, N=64, K=64)
   const uint32_t o = x.tmem + ((c & 1) ? TM_OA : TM_OB);
 #pragma unroll
@@ -324,7 +346,12 @@ __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   umma_commit(&x.bars[B_CKFREE + (c & 1)]);
 }
 // U^T = V^T (T beta)^T   (M=128 value columns, N=64, K=64); v read as MN-major A
+template <bool LEAN>
 __device__ __forceinline__ void issue_u(const Ctx& x) {
+  if (LEAN && x.v_zero) {   // U = 0: nothing to compute (the Delta product starts from zero)
+    umma_commit(&x.bars[B_UDONE]);
+    return;
+  }
   tc_fence_after();
   const uint32_t sbase = smem_u32(x.sm);
   const uint32_t tb = sbase + OFF_TB, vv = sbase + OFF_V;
@@ -491,6 +518,7 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, i
   return true;
 }
 
+template <bool LEAN>
 __device__ void prep_a_role(const Ctx& x, const Args& p) {
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
@@ -582,7 +610,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
         uint2* kp = reinterpret_cast<uint2*>(kq + koff + kb * 16384 + swz128(r * 128 + cbyte));
         uint2* qp = reinterpret_cast<uint2*>(kq + qoff + kb * 16384 + swz128(r * 128 + cbyte));
         const uint2 kr = valid ? *kp : make_uint2(0u, 0u);
-        const uint2 qv = valid ? *qp : make_uint2(0u, 0u);
+        const uint2 qv = (valid && !LEAN) ? *qp : make_uint2(0u, 0u);
         float e[4], f[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -591,7 +619,8 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
         }
         const uint32_t e01 = pack_bf16(e[0], e[1]), e23 = pack_bf16(e[2], e[3]);
         *kp = make_uint2(mul_bf16x2(kr.x, e01), mul_bf16x2(kr.y, e23));
-        *qp = make_uint2(mul_bf16x2(qv.x, e01), mul_bf16x2(qv.y, e23));
+        if (!LEAN)   // Rq only where there is an output
+          *qp = make_uint2(mul_bf16x2(qv.x, e01), mul_bf16x2(qv.y, e23));
         if (ok)
           *reinterpret_cast<uint2*>(ck + kb * 8192 + swz128(r * 128 + cbyte)) =
               make_uint2(mul_bf16x2(kr.x, pack_bf16(f[0], f[1])),
@@ -687,6 +716,7 @@ __device__ __forceinline__ void issue_gram(const Ctx& x, int g) {
   umma_commit(&x.bars[B_GRAM]);
 }
 
+template <bool LEAN>
 __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
                             const CUtensorMap* map_la) {
   const int tid = threadIdx.x - PB_WARP0 * 32;
@@ -712,7 +742,7 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
         const uint32_t par = ((cn - 3) / 3) & 1;
         if (block ? !wait_b(x, B_KQFREE + cn % 3, par) : !mbar_test_wait(fb, par)) return;
       }
-      issue_kq(x, map_k, map_q, cn);
+      issue_kq<LEAN>(x, map_k, map_q, cn);
       if (cn + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
       ++kq_issued;
     }
@@ -766,7 +796,7 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
             o4.w = (col0 + m + 3 < r) ? br * v[m + 3] : 0.f;
             *reinterpret_cast<float4*>(&aw[r * AW + col0 + m]) = o4;
           }
-        } else {
+        } else if (!LEAN) {   // (P only where there is an output)
           uint8_t* pt = ck + 16384;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -975,6 +1005,7 @@ __device__ __noinline__ void st_store_ragged(uint32_t lane_addr, __nv_bfloat16* 
 // state warps (12-19): the sequential pass over chunks. Thread = (TMEM lane j =
 // value column, half hh of the key channels / of the chunk rows).
 // ============================================================================
+template <bool LEAN>
 __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v,
                            const CUtensorMap* map_o) {
   const int tid = threadIdx.x - ST_WARP0 * 32;
@@ -989,9 +1020,11 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 
   // ---- prologue: the fp32 state (h0, identity or zeros) and cleared output accumulators
   st_load_state(x.tmem + TM_S + lb, x.h0, x.h0_identity, j, 64 * hh);
-  tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
-  tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
-  tmem_st_wait();
+  if (!LEAN) {
+    tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
+    tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
+    tmem_st_wait();
+  }
   if (x.v_zero) {   // a zero v tile for every chunk (U = 0)
     for (int i = tid; i < 1024; i += ST_THREADS)
       *reinterpret_cast<uint4*>(x.sm + OFF_V + i * 16) = make_uint4(0u, 0u, 0u, 0u);
@@ -1042,7 +1075,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       return true;   // not ready yet: issued later, before the chunk's [O | Delta] product
     }
     v_landed = cu + 1;
-    issue_u(x);
+    issue_u<LEAN>(x);
     u_issued = cu + 1;
     return true;
   };
@@ -1079,7 +1112,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     if (issuer && alive) {
       mbar_arrive(&x.bars[B_WREAD]);
       alive = issue_u_of(0, true);
-      if (alive) issue_crit(x, 0);
+      if (alive) issue_crit<LEAN>(x, 0);
     }
   }
   for (int c = 0; c < n; ++c) {
@@ -1109,7 +1142,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     }
     named_bar_sync(BAR_ST, ST_THREADS);
     if (issuer && alive) {
-      issue_update(x, c);
+      issue_update<LEAN>(x, c);
       if (c + 1 < n) alive = issue_u_of(c + 1, false);
     }
     // ---- next chunk's decayed state, as soon as this chunk's update has landed
@@ -1125,10 +1158,11 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       if (issuer && alive) {
         mbar_arrive(&x.bars[B_WREAD]);
         if (u_issued < c + 2) alive = issue_u_of(c + 1, true);
-        if (alive) issue_crit(x, c + 1);
+        if (alive) issue_crit<LEAN>(x, c + 1);
       }
     }
     // ---- output of chunk c (off the sequential path), then clear its columns
+    if (LEAN) continue;
     alive = alive && wait_b(x, B_PD, c & 1);
     if (alive) {
       tc_fence_after();
@@ -1179,6 +1213,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 // ============================================================================
 // kernel: one CTA per (sequence, head)
 // ============================================================================
+template <bool LEAN>
 __global__ void __launch_bounds__(THREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_la,
@@ -1264,11 +1299,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.tmem = *tmem_slot;
 
   if (warp < PA_WARPS) {
-    prep_a_role(x, args);
+    prep_a_role<LEAN>(x, args);
   } else if (warp < ST_WARP0) {
-    prep_b_role(x, &map_k, &map_q, &map_la);
+    prep_b_role<LEAN>(x, &map_k, &map_q, &map_la);
   } else {
-    state_role(x, args, &map_v, &map_o);
+    state_role<LEAN>(x, args, &map_v, &map_o);
   }
   tc_fence_before();
   __syncthreads();

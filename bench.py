@@ -38,6 +38,12 @@ D = 128
 PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * D + 4 * D + 4 + 2 * D   # q,k,v bf16 + log_alpha f32 + beta + o
 STATE_BYTES = 4 * D * D
 DECODE_BYTES_PER_CHAIN = 2 * STATE_BYTES + 4 * 2 * D + 2 + 2 * D   # state rw + q,k,v,la + beta + o
+DECODE_TOKENS = 4   # tokens per sequence per call of the multi-token decode step
+
+
+def decode_tokens_bytes_per_chain(t: int) -> int:
+    """State read + write once, plus q, k, v, log_alpha, beta and o of t tokens (bf16)."""
+    return 2 * STATE_BYTES + t * (4 * 2 * D + 2 + 2 * D)
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -313,6 +319,29 @@ def time_decode(kda, dec, steps, warmup, stream):
     return a.elapsed_time(b)
 
 
+def time_decode_tokens(kda, pool, state, calls, warmup, stream):
+    """kda_decode_tokens calls over a pool of distinct [N, t, H, 128] input sets; the
+    state is updated in place by every call."""
+    n_avail = len(pool)
+    o = torch.empty_like(pool[0]["q"])
+
+    def call(c):
+        x = pool[c % n_avail]
+        kda.decode_tokens(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], state, o=o)
+
+    for c in range(warmup):
+        call(c)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for c in range(calls):
+        call(c)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
 def time_e2e(kda, inp, steps, stream):
     """Public API with host buffers: H2D of the step's inputs from pinned memory,
     the prefill, and D2H of its outputs (o and the final state), every step."""
@@ -414,7 +443,19 @@ def main():
     # whole-job bytes per step (every replica moves its own states) over the slowest rank
     dec_gbs = replica_throughput(float(chains * DECODE_BYTES_PER_CHAIN * args.decode_steps),
                                  dec_ms, ws) / 1e9
-    del dec
+    # multi-token decode: DECODE_TOKENS consecutive steps of every sequence per call,
+    # inputs grouped from the same draws (sequence-major), the same state in place
+    t_dec = DECODE_TOKENS
+    pool = [{n: dec[n][i * t_dec:(i + 1) * t_dec].transpose(0, 1).contiguous()
+             for n in ("q", "k", "v", "log_alpha", "beta")} for i in range(n_pool // t_dec)]
+    dt_calls = max(1, args.decode_steps // t_dec)
+    _barrier(ws)
+    dt_ms = _max_over_ranks(time_decode_tokens(kda, pool, dec["state"], dt_calls, args.warmup,
+                                               stream), ws)
+    dt_bytes = chains * decode_tokens_bytes_per_chain(t_dec)
+    dt_gbs = replica_throughput(float(dt_bytes * dt_calls), dt_ms, ws) / 1e9
+    dt_tok_s = replica_throughput(float(dcfg.n_seqs * t_dec * dt_calls), dt_ms, ws)
+    del dec, pool
     torch.cuda.empty_cache()
 
     # ---- end to end through the public API with host buffers
@@ -464,6 +505,15 @@ def main():
                                     "algorithmic_bytes_per_step": chains * DECODE_BYTES_PER_CHAIN},
                        "gpu_launches": args.decode_steps,
                        "l2": "state 512 MiB > L2"},
+            "decode_tokens": {"workload": f"{dcfg.name}_t{t_dec}", "calls": dt_calls,
+                              "tokens_per_call": t_dec,
+                              "us_per_call": dt_ms / dt_calls * 1e3,
+                              "tokens_per_s": dt_tok_s, "GBps": dt_gbs,
+                              "roofline": {"bound": "hbm", "achieved": dt_gbs, "peak": hbm_peak,
+                                           "unit": "GB/s", "frac": dt_gbs / (hbm_peak * ws),
+                                           "algorithmic_bytes_per_call": dt_bytes},
+                              "gpu_launches": dt_calls,
+                              "l2": "state 512 MiB > L2"},
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

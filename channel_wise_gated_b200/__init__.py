@@ -7,6 +7,7 @@ check their dtypes, shapes and contiguity, and pass raw pointers through.
 
     o, hT = chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None)
     o     = decode_step(q, k, v, log_alpha, beta, state)      # state updated in place
+    o     = decode_tokens(q, k, v, log_alpha, beta, state)    # t tokens per sequence
 """
 
 from __future__ import annotations
@@ -137,6 +138,38 @@ def decode_step(q, k, v, log_alpha, beta, state, o=None):
     st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state),
                              _ptr(o), N, H, _DT[q.dtype], _DT[log_alpha.dtype], _stream_ptr(dev))
     _native.check(st, "kda_decode_step")
+    return o
+
+
+def decode_tokens(q, k, v, log_alpha, beta, state, o=None):
+    """Several recurrent KDA steps per (sequence, head) in one call, state in place.
+
+    q, k, v: [N, t, H, 128] bf16 or fp32 (sequence-major, t = 1..16 new tokens per
+    sequence); log_alpha: [N, t, H, 128] and beta: [N, t, H] (bf16 or fp32, same
+    dtype); state: [N, H, 128, 128] fp32, read once and written once. Returns o like q.
+    """
+    lib = _native.load()
+    if q.dim() != 4 or q.shape[3] != D:
+        raise ValueError("q must be [N, t, H, 128]")
+    N, t, H, _ = q.shape
+    if not 1 <= t <= _native.KDA_DECODE_MAX_TOKENS:
+        raise ValueError(f"t must be in 1..{_native.KDA_DECODE_MAX_TOKENS}")
+    dev = q.device
+    if q.dtype not in _DT or log_alpha.dtype not in _DT:
+        raise TypeError("unsupported dtype")
+    for name, x in (("q", q), ("k", k), ("v", v)):
+        _need(x, name, q.dtype, (N, t, H, D), dev)
+    _need(log_alpha, "log_alpha", log_alpha.dtype, (N, t, H, D), dev)
+    _need(beta, "beta", log_alpha.dtype, (N, t, H), dev)
+    _need(state, "state", torch.float32, (N, H, D, D), dev)
+    if o is None:
+        o = torch.empty_like(q)
+    else:
+        _need(o, "o", q.dtype, (N, t, H, D), dev)
+    st = lib.kda_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                               _ptr(state), _ptr(o), N, t, H, _DT[q.dtype], _DT[log_alpha.dtype],
+                               _stream_ptr(dev))
+    _native.check(st, "kda_decode_tokens")
     return o
 
 

@@ -248,6 +248,19 @@ int launch_decode(const void* q, const void* k, const void* v, const void* log_a
   return launch_status();
 }
 
+template <typename TQ, typename TG>
+int launch_decode_tokens(const void* q, const void* k, const void* v, const void* log_alpha,
+                         const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_tokens,
+                         int32_t n_heads, cudaStream_t stream) {
+  const unsigned chains = (unsigned)n_seqs * (unsigned)n_heads;
+  kda::kda_decode_tokens_kernel<TQ, TG><<<chains, kda::DEC_THREADS, 0, stream>>>(
+      static_cast<const TQ*>(q), static_cast<const TQ*>(k), static_cast<const TQ*>(v),
+      static_cast<const TG*>(log_alpha), static_cast<const TG*>(beta), state, static_cast<TQ*>(o),
+      n_heads, n_tokens);
+  return launch_status();
+}
+static_assert(KDA_DECODE_MAX_TOKENS == kda::DEC_MAX_TOKENS, "token limit of the ABI and the kernel");
+
 // Device address of g_kda_static_scratch on the current device. In host code the
 // array's name only stands in for the symbol, so the address is looked up once per
 // device, with that device current, and kept.
@@ -368,6 +381,34 @@ int kda_decode_step(const void* q, const void* k, const void* v, const void* log
     return launch_decode<float, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o, n_seqs,
                                                n_heads, stream);
   return launch_decode<float, float>(q, k, v, log_alpha, beta, state, o, n_seqs, n_heads, stream);
+}
+
+int kda_decode_tokens(const void* q, const void* k, const void* v, const void* log_alpha,
+                      const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_tokens,
+                      int32_t n_heads, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                      cudaStream_t stream) {
+  if ((qkv_dtype != KDA_F32 && qkv_dtype != KDA_BF16) ||
+      (gate_dtype != KDA_F32 && gate_dtype != KDA_BF16))
+    return KDA_ERR_DTYPE;
+  if (n_seqs <= 0 || n_heads <= 0 || n_tokens <= 0 || n_tokens > KDA_DECODE_MAX_TOKENS ||
+      (int64_t)n_seqs * n_heads > (int64_t)INT32_MAX)
+    return KDA_ERR_SHAPE;
+  if (!q || !k || !v || !log_alpha || !beta || !state || !o) return KDA_ERR_NULL;
+  const void* ptrs[] = {q, k, v, log_alpha, state, o};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return KDA_ERR_ALIGN;
+  if (qkv_dtype == KDA_BF16) {
+    if (gate_dtype == KDA_BF16)
+      return launch_decode_tokens<__nv_bfloat16, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o,
+                                                                n_seqs, n_tokens, n_heads, stream);
+    return launch_decode_tokens<__nv_bfloat16, float>(q, k, v, log_alpha, beta, state, o, n_seqs,
+                                                      n_tokens, n_heads, stream);
+  }
+  if (gate_dtype == KDA_BF16)
+    return launch_decode_tokens<float, __nv_bfloat16>(q, k, v, log_alpha, beta, state, o, n_seqs,
+                                                      n_tokens, n_heads, stream);
+  return launch_decode_tokens<float, float>(q, k, v, log_alpha, beta, state, o, n_seqs, n_tokens,
+                                            n_heads, stream);
 }
 
 int kda_device_status(cudaStream_t stream) {

@@ -111,3 +111,113 @@ kda_decode_step_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const
 }
 
 }  // namespace kda
+
+namespace kda {
+
+// Several consecutive tokens per (sequence, head) in one pass over the state: the
+// recurrence of section 3 applied n_tokens times, with the state read once before the
+// first token and written once after the last (speculative or multi-token decoding,
+// where a few new tokens per sequence are verified at once). Per token the arithmetic
+// is the single step's above, in the same order, so the result equals n_tokens
+// consecutive single steps. Inputs are packed sequence-major like a prefill batch of
+// equal lengths: [n_seqs, n_tokens, n_heads, 128] (beta [n_seqs, n_tokens, n_heads]).
+// All tokens' inputs are staged in shared memory up front, their loads in flight
+// together with the state's.
+constexpr int DEC_MAX_TOKENS = 16;
+
+template <typename TQ, typename TG>
+__global__ void __launch_bounds__(DEC_THREADS, 2)
+kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
+                         const TQ* __restrict__ v, const TG* __restrict__ log_alpha,
+                         const TG* __restrict__ beta, float* __restrict__ state,
+                         TQ* __restrict__ o, int n_heads, int n_tokens) {
+  const int chain = blockIdx.x;          // (sequence, head) flattened, as the state
+  const int seq = chain / n_heads, h = chain - seq * n_heads;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  __shared__ float s_k[DEC_MAX_TOKENS][D], s_q[DEC_MAX_TOKENS][D];
+  __shared__ float s_a[DEC_MAX_TOKENS][D], s_v[DEC_MAX_TOKENS][D];
+  __shared__ float4 s_u[DEC_THREADS / 32][32], s_y[DEC_THREADS / 32][32];
+  __shared__ float s_beta[DEC_MAX_TOKENS];
+
+  float4* S = reinterpret_cast<float4*>(state + (size_t)chain * D * D);
+  const int row0 = warp * DEC_ROWS_PER_WARP;
+
+  float4 s[DEC_ROWS_PER_WARP];
+#pragma unroll
+  for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) s[i] = __ldcs(&S[(row0 + i) * (D / 4) + lane]);
+
+#pragma unroll 1
+  for (int i = tid; i < n_tokens * D; i += DEC_THREADS) {
+    const int t = i / D, c = i - t * D;
+    const size_t base = (((size_t)seq * n_tokens + t) * n_heads + h) * D + c;
+    s_k[t][c] = to_f32(k[base]);
+    s_q[t][c] = to_f32(q[base]);
+    s_v[t][c] = to_f32(v[base]);
+    s_a[t][c] = expf(to_f32(log_alpha[base]));
+  }
+  if (tid < n_tokens) s_beta[tid] = to_f32(beta[((size_t)seq * n_tokens + tid) * n_heads + h]);
+  // this lane's 4 output columns of token 0; one token further is n_heads * D elements
+  TQ* od = o + ((size_t)seq * n_tokens * n_heads + h) * D + lane * 4;
+  const size_t o_step = (size_t)n_heads * D;
+  __syncthreads();
+
+#pragma unroll 1
+  for (int t = 0; t < n_tokens; ++t, od += o_step) {
+    // decay and the two partial projections over this warp's rows
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) {
+      const int r = row0 + i;
+      const float a = s_a[t][r], kr = s_k[t][r], qr = s_q[t][r];
+      s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+      u.x = fmaf(kr, s[i].x, u.x); u.y = fmaf(kr, s[i].y, u.y);
+      u.z = fmaf(kr, s[i].z, u.z); u.w = fmaf(kr, s[i].w, u.w);
+      y.x = fmaf(qr, s[i].x, y.x); y.y = fmaf(qr, s[i].y, y.y);
+      y.z = fmaf(qr, s[i].z, y.z); y.w = fmaf(qr, s[i].w, y.w);
+    }
+    s_u[warp][lane] = u;
+    s_y[warp][lane] = y;
+
+    float kq = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) kq = fmaf(s_k[t][lane * 4 + i], s_q[t][lane * 4 + i], kq);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    __syncthreads();
+
+    u = make_float4(0.f, 0.f, 0.f, 0.f);
+    y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < DEC_THREADS / 32; ++w) {
+      const float4 a = s_u[w][lane], b = s_y[w][lane];
+      u.x += a.x; u.y += a.y; u.z += a.z; u.w += a.w;
+      y.x += b.x; y.y += b.y; y.z += b.z; y.w += b.w;
+    }
+    const float bt = s_beta[t];
+    const float4 vv = reinterpret_cast<const float4*>(s_v[t])[lane];
+    float4 dl;
+    dl.x = bt * (vv.x - u.x); dl.y = bt * (vv.y - u.y);
+    dl.z = bt * (vv.z - u.z); dl.w = bt * (vv.w - u.w);
+
+    if (warp == 0) {
+      od[0] = from_f32<TQ>(fmaf(kq, dl.x, y.x));
+      od[1] = from_f32<TQ>(fmaf(kq, dl.y, y.y));
+      od[2] = from_f32<TQ>(fmaf(kq, dl.z, y.z));
+      od[3] = from_f32<TQ>(fmaf(kq, dl.w, y.w));
+    }
+#pragma unroll
+    for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) {
+      const float kr = s_k[t][row0 + i];
+      s[i].x = fmaf(kr, dl.x, s[i].x); s[i].y = fmaf(kr, dl.y, s[i].y);
+      s[i].z = fmaf(kr, dl.z, s[i].z); s[i].w = fmaf(kr, dl.w, s[i].w);
+    }
+    __syncthreads();   // s_u / s_y are rewritten by the next token
+  }
+#pragma unroll
+  for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) __stcs(&S[(row0 + i) * (D / 4) + lane], s[i]);
+}
+
+}  // namespace kda

@@ -209,6 +209,33 @@ int kda_decode_step(const void* q, const void* k, const void* v, const void* log
                     kda_dtype qkv_dtype, kda_dtype gate_dtype, cudaStream_t stream);
 
 /*
+ * kda_decode_tokens - n_tokens consecutive recurrent KDA updates per (sequence,
+ * head), in place, reading the state once and writing it once.
+ *
+ * The same recurrence as kda_decode_step, applied to n_tokens new tokens of every
+ * sequence in order (section 3; section 6.3: generation runs the recurrent form on
+ * the fixed state). It serves multi-token and speculative decoding, where a few
+ * tokens per sequence are processed at once: the state traffic, which dominates a
+ * decode step, is paid once per call instead of once per token. The result equals
+ * n_tokens consecutive kda_decode_step calls.
+ *
+ * Arguments:
+ *   q, k, v     [n_seqs, n_tokens, n_heads, 128], dtype qkv_dtype (sequence-major,
+ *               as a packed prefill batch of equal lengths)
+ *   log_alpha   [n_seqs, n_tokens, n_heads, 128], dtype gate_dtype, entries <= 0
+ *   beta        [n_seqs, n_tokens, n_heads], dtype gate_dtype
+ *   state       [n_seqs, n_heads, 128, 128] fp32, read and overwritten in place
+ *   o           [n_seqs, n_tokens, n_heads, 128] output, dtype qkv_dtype
+ *   n_tokens    1 .. KDA_DECODE_MAX_TOKENS (KDA_ERR_SHAPE otherwise)
+ * Returns KDA_OK or a negative kda_status.
+ */
+#define KDA_DECODE_MAX_TOKENS 16
+int kda_decode_tokens(const void* q, const void* k, const void* v, const void* log_alpha,
+                      const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_tokens,
+                      int32_t n_heads, kda_dtype qkv_dtype, kda_dtype gate_dtype,
+                      cudaStream_t stream);
+
+/*
  * kda_device_status - read and clear the library's device-side error word.
  * Synchronises `stream`. Returns KDA_OK, KDA_ERR_SEQLENS (a kernel saw
  * cu_seqlens that were not monotone or ran past t_total, and clamped them),

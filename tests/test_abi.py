@@ -30,8 +30,8 @@ def lib():
 
 def test_header_declares_expected_entry_points():
     names = declared_functions()
-    for n in ("kda_chunk_fwd", "kda_chunk_fwd_simt", "kda_decode_step", "kda_device_status",
-              "kda_status_string"):
+    for n in ("kda_chunk_fwd", "kda_chunk_fwd_simt", "kda_decode_step", "kda_decode_tokens",
+              "kda_device_status", "kda_status_string"):
         assert n in names
 
 
@@ -108,6 +108,27 @@ def test_decode_validation(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 2, bf, bf, None) == _native.KDA_ERR_SHAPE
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 3, bf, None) == _native.KDA_ERR_DTYPE
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, FAKE, 4, 2, bf, bf, None) == _native.KDA_ERR_ALIGN
+
+
+def test_decode_tokens_validation(lib):
+    f = lib.kda_decode_tokens
+    bf = _native.KDA_BF16
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert f(None, *ok[1:], 4, 2, 2, bf, bf, None) == _native.KDA_ERR_NULL
+    assert f(*ok[:5], None, FAKE, 4, 2, 2, bf, bf, None) == _native.KDA_ERR_NULL
+    assert f(*ok, 0, 2, 2, bf, bf, None) == _native.KDA_ERR_SHAPE
+    assert f(*ok, 4, 0, 2, bf, bf, None) == _native.KDA_ERR_SHAPE
+    assert f(*ok, 4, _native.KDA_DECODE_MAX_TOKENS + 1, 2, bf, bf, None) == _native.KDA_ERR_SHAPE
+    assert f(*ok, 4, 2, 0, bf, bf, None) == _native.KDA_ERR_SHAPE
+    assert f(*ok, 4, 2, 2, 5, bf, None) == _native.KDA_ERR_DTYPE
+    assert f(*ok, 4, 2, 2, bf, 9, None) == _native.KDA_ERR_DTYPE
+    assert f(*ok[:5], FAKE + 4, FAKE, 4, 2, 2, bf, bf, None) == _native.KDA_ERR_ALIGN
+
+
+def test_decode_token_limit_matches_header():
+    text = open(HEADER).read()
+    m = re.search(r"#define KDA_DECODE_MAX_TOKENS (\d+)", text)
+    assert m and int(m.group(1)) == _native.KDA_DECODE_MAX_TOKENS
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -47,12 +47,20 @@ def decode_tokens_bytes_per_chain(t: int) -> int:
 L2_BYTES = 126 * 1024 * 1024
 
 
+# The sources that make up the profiled prefill path: the chunk kernel, its sm_100a
+# building blocks, the segment scan, and the file that builds its tensor maps and
+# launches it (plus the ABI header). The decode and fp32 kernels live in files of
+# their own and do not enter.
+CHUNK_KERNEL_SOURCES = ("kda_api.cu", "kda_chunk_tc.cuh", "kda_common.cuh", "kda_segment.cuh",
+                        "kda_sm100.cuh")
+
+
 def _source_hash() -> str:
-    """sha256 prefix of the kernel sources (csrc/*.cu, csrc/*.cuh, include/kda.h)."""
-    import glob
+    """sha256 prefix of the prefill chunk kernel's sources (CHUNK_KERNEL_SOURCES and
+    include/kda.h): the ncu figures in profiles/ hold while it is unchanged."""
     import hashlib
     csrc = os.path.join(ROOT, "channel_wise_gated_b200", "csrc")
-    files = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")))
+    files = [os.path.join(csrc, f) for f in sorted(CHUNK_KERNEL_SOURCES)]
     files.append(os.path.join(ROOT, "include", "kda.h"))
     h = hashlib.sha256()
     for f in files:

@@ -252,12 +252,11 @@ template <typename TQ, typename TG>
 int launch_decode_tokens(const void* q, const void* k, const void* v, const void* log_alpha,
                          const void* beta, float* state, void* o, int32_t n_seqs, int32_t n_tokens,
                          int32_t n_heads, cudaStream_t stream) {
-  const unsigned chains = (unsigned)n_seqs * (unsigned)n_heads;
-  kda::kda_decode_tokens_kernel<TQ, TG><<<chains, kda::DEC_THREADS, 0, stream>>>(
+  const cudaError_t e = kda::launch_decode_tokens<TQ, TG>(
       static_cast<const TQ*>(q), static_cast<const TQ*>(k), static_cast<const TQ*>(v),
       static_cast<const TG*>(log_alpha), static_cast<const TG*>(beta), state, static_cast<TQ*>(o),
-      n_heads, n_tokens);
-  return launch_status();
+      n_seqs, n_tokens, n_heads, stream);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 static_assert(KDA_DECODE_MAX_TOKENS == kda::DEC_MAX_TOKENS, "token limit of the ABI and the kernel");
 

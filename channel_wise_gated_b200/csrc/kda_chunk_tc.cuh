@@ -32,6 +32,7 @@
 //   W'^T = -Rk^T (T beta)^T               (the -W' tile is written from it)
 // TMEM (512 columns):   0 S^T fp32 | 128 S''^T bf16 pairs | 192 O (odd chunks) |
 //   256 U then Delta | 320 O (even chunks) | 384 Gram [A;P] | 448 -W'^T
+//   (Delta^T is read out of 256-319 and written back there as bf16 pairs)
 // The stacked B operand alternates [-W' ; Rq] (even chunks) and [Rq ; -W'] (odd)
 // so that Delta always lands in columns 256-319 while the output alternates
 // between the two regions around it: the output of chunk c is read while chunk
@@ -43,8 +44,9 @@
 //               thread issues the Gram and W' products, the k/q TMA loads and the L2
 //               prefetch of the log-decay
 //   warps 12-19 state  (chunk c):   decay S in TMEM and write S'', the -W' tile, Delta
-//               tile, output;
-//               its first thread issues the state products, U and the v TMA loads
+//               as bf16 pairs back into TMEM (the A operand of the update), the
+//               output tile; its first thread issues the state products, U, the v
+//               TMA loads and the output's TMA store
 // Every mbarrier wait is bounded; a timeout flags KDA_ERR_TIMEOUT and every role
 // leaves (a group keeps meeting at its own named barriers, doing no work).
 #pragma once
@@ -67,6 +69,7 @@ constexpr int PB_THREADS = 128;
 constexpr int ST_THREADS = ST_WARPS * 32;
 static_assert(PB_WARP0 % 4 == 0 && ST_WARP0 % 4 == 0, "TMEM lane quarters follow warp % 4");
 constexpr uint32_t BAR_PA = 1, BAR_PB = 2, BAR_ST = 3;   // named barriers (0 is __syncthreads)
+constexpr uint32_t BAR_OUT = 4;   // state warps: output tile staged (arrive), then stored
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float GUARD_LOG2 = 60.0f * 1.4426950408889634f;
 constexpr uint64_t WAIT_NS = 2000000000ull;
@@ -81,7 +84,7 @@ constexpr uint32_t OFF_KQ = 0;
 constexpr uint32_t OFF_CKP = OFF_KQ + 3 * KQ_BYTES;
 constexpr uint32_t OFF_V = OFF_CKP + 2 * CKP_BYTES;   // v [2 column blocks][64][128 B]
 constexpr uint32_t OFF_TB = OFF_V + 16384;            // T*beta [64 r][64 i] bf16, K-major
-constexpr uint32_t OFF_DT = OFF_TB + 8192;            // Delta^T [128 j][64 r] bf16, K-major
+constexpr uint32_t OFF_DT = OFF_TB + 8192;            // output staging [64 rows][128 cols] bf16
 constexpr int AW = 68;                                // fp32 pitch of the A / T workspace
 constexpr uint32_t OFF_AW = OFF_DT + 16384;           // also the exact path's staging area
 constexpr uint32_t OFF_XS = OFF_AW + 64 * AW * 4;     // 6 extra 16x16 fp32 blocks
@@ -103,7 +106,7 @@ static_assert(64 * 64 * 4 <= 64 * AW * 4, "exact-path staging of one channel hal
 constexpr uint32_t TM_S = 0;      // S^T fp32 master: lane = value column, column = key channel
 constexpr uint32_t TM_SB = 128;   // S''^T bf16, two channels per column (the A operand)
 constexpr uint32_t TM_OA = 192;   // O^T of odd chunks
-constexpr uint32_t TM_D = 256;    // U^T, then Delta^T
+constexpr uint32_t TM_D = 256;    // U^T, then Delta^T fp32, then its bf16 pairs (see dpair_col)
 constexpr uint32_t TM_OB = 320;   // O^T of even chunks
 constexpr uint32_t TM_G = 384;    // Gram [A;P] or [P;A] (M=128, N=64)
 constexpr uint32_t TM_W = 448;    // -W'^T (M=128 channels, N=64 rows)
@@ -320,18 +323,23 @@ __device__ __forceinline__ void issue_crit(const Ctx& x, int c) {
   umma_commit(&x.bars[B_CRIT]);
   umma_commit(&x.bars[B_KQFREE + c % 3]);
 }
-// S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T (not without output)
+// TMEM column of the bf16 Delta^T pairs of K step kk (chunk rows 16kk..16kk+15): the
+// state warps write rows 0-31 into the first 16 columns of the Delta region and rows
+// 32-63 into its last 16, each warp inside the columns it has just read
+__device__ __forceinline__ uint32_t dpair_col(int kk) { return TM_D + (kk < 2 ? 8 * kk : 48 + 8 * (kk - 2)); }
+
+// S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T (not without output);
+// Delta^T is the A operand, read from TMEM
 template <bool LEAN>
 __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   tc_fence_after();
   const uint32_t sbase = smem_u32(x.sm);
-  const uint32_t dt = sbase + OFF_DT;
   const uint32_t ck = sbase + OFF_CKP + (c & 1) * CKP_BYTES;
   // (M=128, N=128, K=64); Ck read as an MN-major B operand
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk)
-    umma_bf16(x.tmem + TM_S, kdesc128(dt + kk * 32), make_sdesc(ck + kk * 2048, 8192, 1024, SWZ_128B),
-              IDESC_Z, 1u);
+    umma_bf16_tmem_a(x.tmem + TM_S, x.tmem + dpair_col(kk),
+                     make_sdesc(ck + kk * 2048, 8192, 1024, SWZ_128B), IDESC_Z, 1u);
   umma_commit(&x.bars[B_ZDONE]);
   if (LEAN) {
     umma_commit(&x.bars[B_CKFREE + (c & 1)]);
@@ -341,7 +349,7 @@ __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   const uint32_t o = x.tmem + ((c & 1) ? TM_OA : TM_OB);
 #pragma unroll
   for (int kk = 0; kk < 4; ++kk)
-    umma_bf16(o, kdesc128(dt + kk * 32), kdesc128(ck + 16384 + kk * 32), IDESC_PD, 1u);
+    umma_bf16_tmem_a(o, x.tmem + dpair_col(kk), kdesc128(ck + 16384 + kk * 32), IDESC_PD, 1u);
   umma_commit(&x.bars[B_PD]);
   umma_commit(&x.bars[B_CKFREE + (c & 1)]);
 }
@@ -1118,28 +1126,28 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   for (int c = 0; c < n; ++c) {
     const int64_t t0 = x.bos + (int64_t)c * CHUNK;
     const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
-    // ---- Delta^T (TMEM) -> bf16 tile rows j, chunk rows 32hh..32hh+31. The tile
-    //      held the previous chunk's output on its way out: the store must have read it.
+    // ---- Delta^T fp32 (TMEM, chunk rows 32hh..32hh+31 of lane j) -> bf16 pairs in the
+    //      same lanes, inside the columns just read: the A operand of the update
     alive = alive && wait_b(x, B_CRIT, c & 1);
-    if (c > 0) {
-      if (issuer) bulk_wait_read_all();
-      named_bar_sync(BAR_ST, ST_THREADS);
-    }
     if (alive) {
       tc_fence_after();
       float v[32];
       tmem_ld32(x.tmem + TM_D + lb + 32 * hh, v);
       tmem_ld_wait();
+      uint32_t pk[16];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch)
-        *reinterpret_cast<uint4*>(dt + swz128(j * 128 + 64 * hh + 16 * ch)) = pack8(v + 8 * ch);
-      fence_proxy_async_smem();
+      for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+      tmem_st16(x.tmem + TM_D + lb + 48 * hh, pk);
+      tmem_st_wait();
       tc_fence_before();
       if (issuer && c + 1 < n) {   // U(c) is done: v of the next chunk may land
         issue_v(x, map_v, c + 1);
         v_issued = c + 2;
       }
     }
+    // (the output tile of the previous chunk must have been read by its store before
+    //  anyone stages this chunk's output in it: every warp passes this barrier first)
+    if (issuer && c > 0) bulk_wait_read_all();
     named_bar_sync(BAR_ST, ST_THREADS);
     if (issuer && alive) {
       issue_update<LEAN>(x, c);
@@ -1170,7 +1178,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       if (!x.write_o) {
         // (segment state pass: no output)
       } else if (L == CHUNK) {
-        // full chunk: into the (now free) Delta^T tile in the o tile layout, then one
+        // full chunk: into the output tile (its previous store has read it), then one
         // TMA store of [64 rows][128 columns]
         float v[32];
         tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
@@ -1191,7 +1199,13 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       tc_fence_before();
     }
     if (L == CHUNK && x.write_o) {
-      named_bar_sync(BAR_ST, ST_THREADS);
+      // the warps that do not issue only report their part staged and move on to the
+      // next chunk; the issuing warp waits for all parts and sends the tile
+      if (sw != 0) {
+        named_bar_arrive(BAR_OUT, ST_THREADS);
+        continue;
+      }
+      named_bar_sync(BAR_OUT, ST_THREADS);
       if (issuer && alive) {
         tma_store_2d(map_o, dt, x.h * D, (int)t0);
         tma_store_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);

@@ -220,4 +220,15 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
   for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) __stcs(&S[(row0 + i) * (D / 4) + lane], s[i]);
 }
 
+// Host side: one CTA per (sequence, head); returns the launch's CUDA error.
+template <typename TQ, typename TG>
+cudaError_t launch_decode_tokens(const TQ* q, const TQ* k, const TQ* v, const TG* log_alpha,
+                                 const TG* beta, float* state, TQ* o, int n_seqs, int n_tokens,
+                                 int n_heads, cudaStream_t stream) {
+  const unsigned chains = (unsigned)n_seqs * (unsigned)n_heads;
+  kda_decode_tokens_kernel<TQ, TG><<<chains, DEC_THREADS, 0, stream>>>(q, k, v, log_alpha, beta,
+                                                                       state, o, n_heads, n_tokens);
+  return cudaGetLastError();
+}
+
 }  // namespace kda

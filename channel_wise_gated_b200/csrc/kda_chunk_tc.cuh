@@ -41,12 +41,12 @@
 // Roles (640 threads), a pipeline three chunks deep:
 //   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars
 //   warps 8-11  prep B (chunk c+1): Gram readout, UT solve, T*beta tile; its first
-//               thread issues the Gram and W' products, the k/q TMA loads and the L2
+//               thread issues the Gram product, the k/q TMA loads and the L2
 //               prefetch of the log-decay
 //   warps 12-19 state  (chunk c):   decay S in TMEM and write S'', the -W' tile, Delta
 //               as bf16 pairs back into TMEM (the A operand of the update), the
-//               output tile; its first thread issues the state products, U, the v
-//               TMA loads and the output's TMA store
+//               output tile; its first thread issues the state products, W', U, the
+//               v TMA loads and the output's TMA store
 // Every mbarrier wait is bounded; a timeout flags KDA_ERR_TIMEOUT and every role
 // leaves (a group keeps meeting at its own named barriers, doing no work).
 #pragma once
@@ -130,7 +130,6 @@ enum : int {
   B_TB = 10,        // P and T*beta tiles written
   B_WDONE = 11,     // W' MMA done
   B_UDONE = 12,     // U MMA done (v and T*beta free)
-  B_WREAD = 13,     // -W' read out of TMEM (by the state warps)
   B_CRIT = 15,      // [O | Delta] product done
   B_ZDONE = 16,     // state update product done
   B_PD = 17,        // P Delta product done (output complete)
@@ -655,7 +654,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
 }
 
 // ============================================================================
-// prep B (warps 8-11): Gram readout, UT solve, T*beta tile, W' tile
+// prep B (warps 8-11): Gram readout, UT solve, T*beta tile
 // ============================================================================
 
 // acc (two n-halves of a 16x16 C fragment) += X(16x16) * Y(16x16), fp32 blocks in smem.
@@ -818,8 +817,8 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
       tc_fence_before();
     }
     if (tid == 0) push_kq(c + 2, false);
-    // the previous chunk's U and W' products must be done reading the T*beta tile (U
-    // may go out before W' completes, from another thread: its commit does not cover W')
+    // the previous chunk's U and W' products must be done reading the T*beta tile (each
+    // has its own commit)
     ok = ok && ((c < 1) || (wait_b(x, B_UDONE, (c - 1) & 1) && wait_b(x, B_WDONE, (c - 1) & 1)));
     if (named_bar_or(BAR_PB, PB_THREADS, !ok)) break;
     // the Gram columns are free again: the next chunk's Gram goes out now if its
@@ -950,9 +949,6 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
     named_bar_sync(BAR_PB, PB_THREADS);
     if (tid == 0) {
       mbar_arrive(&x.bars[B_TB]);
-      // W' of this chunk once the state warps have read out the previous one (they
-      // read it out themselves, right before their [O | Delta] product)
-      if (c == 0 || wait_b(x, B_WREAD, (c - 1) & 1)) issue_w(x, c);
       mbar_arrive(&x.bars[B_WFREE]);   // done with this chunk: the workspace is free
       push_kq(c + 2, false);
     }
@@ -1071,11 +1067,27 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   };
 
   // Thread 0 issues this group's tensor-core products and the v loads. Per chunk:
-  // U (as soon as T*beta and v are there), the [O | Delta] product, then the state
-  // update and P Delta once Delta is in shared memory; the next chunk's v load goes
-  // out once the current U product is done (it precedes [O | Delta] in the pipe).
+  // W' (as soon as T*beta is there, at the latest right before its readout), U (once
+  // v is there too), the [O | Delta] product, then the state update and P Delta once
+  // Delta is back in TMEM; the next chunk's v load goes out once the current U
+  // product is done (it precedes [O | Delta] in the pipe). W' used to be issued by
+  // prep B: an MMA issue holds the issuing thread until the product starts, and
+  // prep B's chain is the one that sets the pace.
   const bool issuer = tid == 0;
   int u_issued = 0, v_issued = 0, v_landed = 0;
+  // W' of chunk cw (from T*beta; the previous W' was read out before the previous
+  // [O | Delta] product, by these warps)
+  int w_issued = 0;
+  auto issue_w_of = [&](int cw, bool block) -> bool {
+    if (block) {
+      if (!wait_b(x, B_TB, cw & 1)) return false;
+    } else if (!mbar_test_wait(&x.bars[B_TB], cw & 1)) {
+      return true;   // not ready yet: issued later, before its readout
+    }
+    issue_w(x, cw);
+    w_issued = cw + 1;
+    return true;
+  };
   auto issue_u_of = [&](int cu, bool block) -> bool {
     if (block) {
       if (!wait_b(x, B_TB, cu & 1) || !wait_b(x, B_VFULL, cu & 1)) return false;
@@ -1115,10 +1127,10 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     }
     alive = wait_b(x, B_TILES + 0, 0);
     if (alive) s_pass(0);
+    if (issuer && alive) alive = issue_w_of(0, true);
     alive = alive && w_readout(0);
     named_bar_sync(BAR_ST, ST_THREADS);
     if (issuer && alive) {
-      mbar_arrive(&x.bars[B_WREAD]);
       alive = issue_u_of(0, true);
       if (alive) issue_crit<LEAN>(x, 0);
     }
@@ -1151,7 +1163,10 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     named_bar_sync(BAR_ST, ST_THREADS);
     if (issuer && alive) {
       issue_update<LEAN>(x, c);
-      if (c + 1 < n) alive = issue_u_of(c + 1, false);
+      if (c + 1 < n) {
+        alive = issue_w_of(c + 1, false);
+        if (alive && w_issued == c + 2) alive = issue_u_of(c + 1, false);
+      }
     }
     // ---- next chunk's decayed state, as soon as this chunk's update has landed
     if (c + 1 < n) {
@@ -1161,10 +1176,10 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         tc_fence_after();
         s_pass(c + 1);
       }
+      if (issuer && alive && w_issued < c + 2) alive = issue_w_of(c + 1, true);
       alive = alive && w_readout(c + 1);
       named_bar_sync(BAR_ST, ST_THREADS);
       if (issuer && alive) {
-        mbar_arrive(&x.bars[B_WREAD]);
         if (u_issued < c + 2) alive = issue_u_of(c + 1, true);
         if (alive) issue_crit<LEAN>(x, c + 1);
       }

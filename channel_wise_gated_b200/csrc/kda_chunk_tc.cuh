@@ -39,10 +39,11 @@
 // c+1 is already accumulating.
 //
 // Roles (640 threads), a pipeline three chunks deep:
-//   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars
+//   warps 0-7   prep A (chunk c+2): cumsum, range guard, Rk/Rq/Ck tiles, scalars;
+//               its first thread issues the Gram product once prep B has read out
+//               the previous one
 //   warps 8-11  prep B (chunk c+1): Gram readout, UT solve, T*beta tile; its first
-//               thread issues the Gram product, the k/q TMA loads and the L2
-//               prefetch of the log-decay
+//               thread issues the k/q TMA loads and the L2 prefetch of the log-decay
 //   warps 12-19 state  (chunk c):   decay S in TMEM and write S'', the -W' tile, Delta
 //               as bf16 pairs back into TMEM (the A operand of the update), the
 //               output tile; its first thread issues the state products, W', U, the
@@ -130,6 +131,8 @@ enum : int {
   B_TB = 10,        // P and T*beta tiles written
   B_WDONE = 11,     // W' MMA done
   B_UDONE = 12,     // U MMA done (v and T*beta free)
+  B_GFREE = 13,     // Gram columns read out (by prep B): the next Gram may go out
+  B_FIN_A = 14,     // drain of prep A's first thread (it issues the Gram)
   B_CRIT = 15,      // [O | Delta] product done
   B_ZDONE = 16,     // state update product done
   B_PD = 17,        // P Delta product done (output complete)
@@ -380,6 +383,26 @@ __device__ __forceinline__ void issue_w(const Ctx& x, int c) {
     umma_bf16(x.tmem + TM_W, make_sdesc(kq + kk * 2048, 16384, 1024, SWZ_128B), kdesc128(tb + kk * 32),
               IDESC_W, kk > 0 ? 1u : 0u);
   umma_commit(&x.bars[B_WDONE]);
+}
+
+// Gram product of chunk g (issued by prep A's first thread once its tiles are written): [A ; P] or [P ; A] =
+// stage tile x Ck^T (M=128, N=64, K=128). For an exact-path chunk only the commit
+// goes out, so the barrier completes one phase per chunk either way.
+__device__ __forceinline__ void issue_gram(const Ctx& x, int g) {
+  const int* xflag = reinterpret_cast<const int*>(x.sm + OFF_XFLAG);
+  if (xflag[g % 3]) {
+    umma_commit(&x.bars[B_GRAM]);
+    return;
+  }
+  tc_fence_after();
+  const uint32_t sbase = smem_u32(x.sm);
+  const uint32_t kq = sbase + OFF_KQ + (g % 3) * KQ_BYTES;
+  const uint32_t ck = sbase + OFF_CKP + (g & 1) * CKP_BYTES;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    umma_bf16(x.tmem + TM_G, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
+              kdesc128(ck + (kk >> 2) * 8192 + (kk & 3) * 32), IDESC_GRAM, kk > 0 ? 1u : 0u);
+  umma_commit(&x.bars[B_GRAM]);
 }
 
 // ============================================================================
@@ -649,12 +672,21 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
     }
     fence_proxy_async_smem();
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
-    if (tid == 0) mbar_arrive(&x.bars[B_TILES + (c & 1)]);
+    if (tid == 0) {
+      mbar_arrive(&x.bars[B_TILES + (c & 1)]);
+      // the Gram product of this chunk, once prep B has read out the previous one. An
+      // MMA issue holds the issuing thread until the product starts; prep A, ahead of
+      // prep B, has the slack for that, prep B does not.
+      if (c == 0 || wait_b(x, B_GFREE, (c - 1) & 1)) issue_gram(x, c);
+    }
   }
+  if (tid == 0) drain(x, B_FIN_A);
 }
 
 // ============================================================================
-// prep B (warps 8-11): Gram readout, UT solve, T*beta tile
+// prep B (warps 8-11): Gram readout, UT solve, T*beta tile (prep B issues no tensor-core
+// product: an MMA issue holds the issuing thread until the product starts, and prep B's
+// chain is the one that sets the pace)
 // ============================================================================
 
 // acc (two n-halves of a 16x16 C fragment) += X(16x16) * Y(16x16), fp32 blocks in smem.
@@ -703,26 +735,6 @@ __device__ __forceinline__ void blk_store_tb(uint8_t* tt, int a, int b, const fl
   }
 }
 
-// Gram product of chunk g (issued by prep B's first thread): [A ; P] or [P ; A] =
-// stage tile x Ck^T (M=128, N=64, K=128). For an exact-path chunk only the commit
-// goes out, so the barrier completes one phase per chunk either way.
-__device__ __forceinline__ void issue_gram(const Ctx& x, int g) {
-  const int* xflag = reinterpret_cast<const int*>(x.sm + OFF_XFLAG);
-  if (xflag[g % 3]) {
-    umma_commit(&x.bars[B_GRAM]);
-    return;
-  }
-  tc_fence_after();
-  const uint32_t sbase = smem_u32(x.sm);
-  const uint32_t kq = sbase + OFF_KQ + (g % 3) * KQ_BYTES;
-  const uint32_t ck = sbase + OFF_CKP + (g & 1) * CKP_BYTES;
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    umma_bf16(x.tmem + TM_G, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
-              kdesc128(ck + (kk >> 2) * 8192 + (kk & 3) * 32), IDESC_GRAM, kk > 0 ? 1u : 0u);
-  umma_commit(&x.bars[B_GRAM]);
-}
-
 template <bool LEAN>
 __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
                             const CUtensorMap* map_la) {
@@ -734,7 +746,6 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
   const int* xflag = reinterpret_cast<const int*>(x.sm + OFF_XFLAG);
   auto A = [&](int a, int b) { return aw + (16 * a) * AW + 16 * b; };
   uint8_t* tt = x.sm + OFF_TB;
-  int gram_issued = 0;   // (thread 0) Gram products issued so far
   // (thread 0) the k/q loads of the CTA: each goes out once its stage slot is free
   // (the [O | Delta] product of the chunk three back done), and prefetches the
   // log-decay of the chunk three later into L2. Polled at a few points of every
@@ -774,11 +785,6 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
     }
     bool ok = wait_b(x, B_TILES + (c & 1), (c >> 1) & 1);
     const bool exact = ok && xflag[s3] != 0;
-    // the Gram of this chunk, unless it went out while the previous chunk was solved
-    if (tid == 0 && ok && c >= gram_issued) {
-      issue_gram(x, c);
-      gram_issued = c + 1;
-    }
     // ---- Gram readout: A rows (beta-scaled, strictly lower) -> fp32 workspace; P -> bf16 tile.
     //      Lanes of the k half hold A, lanes of the q half hold P.
     ok = ok && wait_b(x, B_GRAM, c & 1);
@@ -821,13 +827,8 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
     // has its own commit)
     ok = ok && ((c < 1) || (wait_b(x, B_UDONE, (c - 1) & 1) && wait_b(x, B_WDONE, (c - 1) & 1)));
     if (named_bar_or(BAR_PB, PB_THREADS, !ok)) break;
-    // the Gram columns are free again: the next chunk's Gram goes out now if its
-    // tiles are already written
-    if (tid == 0 && c + 1 < x.n_chunks &&
-        mbar_test_wait(&x.bars[B_TILES + ((c + 1) & 1)], ((c + 1) >> 1) & 1)) {
-      issue_gram(x, c + 1);
-      gram_issued = c + 2;
-    }
+    // the Gram columns are free again: prep A's thread may issue the next Gram
+    if (tid == 0) mbar_arrive(&x.bars[B_GFREE]);
 
     // ---- UT transform: T = (I + A)^{-1}. 16x16 diagonal blocks by forward substitution:
     //      lane j of warp a keeps column j of T_aa in registers (the A values are

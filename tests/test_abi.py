@@ -41,6 +41,40 @@ def test_library_exports_every_declared_symbol(lib):
         assert name in _native.SIGNATURES, f"{name} has no binding signature"
 
 
+def test_every_exported_entry_point_is_declared(lib):
+    """The reverse of the check above: nothing leaves the library under a kda_ name that
+    include/kda.h does not declare (names from the dynamic symbol table of our own build)."""
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    out = subprocess.run([nm, "-D", "--defined-only", _native.LIB_PATH], check=True,
+                         capture_output=True, text=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines()
+                       if ln.split() and ln.split()[-1].startswith("kda_")})
+    assert exported, "no kda_ symbols exported"
+    assert set(exported) <= set(declared_functions()), set(exported) - set(declared_functions())
+
+
+def test_profile_summary_is_machine_readable():
+    """bench.py reads the DRAM traffic per token-head and the kernel-source hash it was
+    taken with from the committed ncu summary; both must parse."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench_mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench_mod)
+    for f in bench_mod.CHUNK_KERNEL_SOURCES:
+        assert os.path.exists(os.path.join(ROOT, "channel_wise_gated_b200", "csrc", f)), f
+    text = open(os.path.join(ROOT, "profiles", "kda_chunk_tc_prefill4k_full.md")).read()
+    mh = re.search(r"^source_hash: ([0-9a-f]{16})$", text, re.M)
+    mb = re.search(r"^split_call_dram_bytes_per_token_head: ([0-9.]+)$", text, re.M)
+    assert mh and mb
+    # at least the algorithmic 1,540 B per token-head, at most a few times it
+    assert 1540 <= float(mb.group(1)) <= 8 * 1540
+    assert re.fullmatch(r"[0-9a-f]{16}", bench_mod._source_hash())
+
+
 def test_status_strings(lib):
     for st in range(0, -9, -1):
         s = _native.status_string(st)

@@ -113,6 +113,20 @@ def chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, o=None, hT=Non
     return o, hT
 
 
+def split_plan(n_heads: int, t_total: int, n_sms: int = 0, workspace_bytes: Optional[int] = None):
+    """Segment bounds of the time split that kda_chunk_fwd_ws uses for one bf16
+    sequence (token offsets, n + 1 of them), or [] when the single pass runs.
+    n_sms = 0 plans for the current device; workspace_bytes None = unlimited."""
+    import ctypes
+    lib = _native.load()
+    bounds = (ctypes.c_int64 * (_native.KDA_MAX_SEGMENTS + 1))()
+    ws = _native.SIZE_MAX if workspace_bytes is None else int(workspace_bytes)
+    n = lib.kda_chunk_fwd_split_plan(int(n_heads), int(t_total), int(n_sms), ws, bounds)
+    if n < 0:
+        raise KdaError(n, "kda_chunk_fwd_split_plan")
+    return [int(bounds[i]) for i in range(n + 1)] if n >= 3 else []
+
+
 def decode_step(q, k, v, log_alpha, beta, state, o=None):
     """One recurrent KDA step per (sequence, head), state updated in place.
 

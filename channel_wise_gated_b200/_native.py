@@ -27,6 +27,8 @@ KDA_ERR_TIMEOUT = -7
 KDA_ERR_SCRATCH = -8
 
 KDA_DECODE_MAX_TOKENS = 16
+KDA_MAX_SEGMENTS = 64
+SIZE_MAX = ctypes.c_size_t(-1).value
 
 # entry point -> argument types (all return int except kda_status_string)
 _P, _I32, _I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
@@ -36,6 +38,7 @@ SIGNATURES = {
     "kda_chunk_fwd_ws": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P,
                          ctypes.c_size_t, _P],
     "kda_chunk_fwd_workspace_size": [_I32, _I64, _I32, ctypes.c_int, ctypes.c_int],
+    "kda_chunk_fwd_split_plan": [_I32, _I64, _I32, ctypes.c_size_t, _P],
     "kda_chunk_fwd_static": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
     "kda_decode_step": [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, ctypes.c_int, ctypes.c_int, _P],
     "kda_decode_tokens": [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, ctypes.c_int, ctypes.c_int,

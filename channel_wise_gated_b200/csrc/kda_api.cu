@@ -16,9 +16,10 @@
 #include "kda_segment.cuh"
 
 // Scratch of kda_chunk_fwd_static, for callers that cannot allocate device memory:
-// a fixed array in every GPU context that loads the library. It covers the time
-// split of any head count on a 148-SM part (at most 220 slots x 64 KiB = 13.75 MiB);
-// larger needs are rejected with KDA_ERR_SCRATCH.
+// a fixed array in every GPU context that loads the library. The time split plans
+// within it (on a 148-SM part the largest plan takes 18.2 MiB of a free workspace,
+// so a few head counts split into fewer segments here); a packed batch's launch
+// order needs 4 bytes per sequence.
 static __device__ __align__(256) unsigned char g_kda_static_scratch[KDA_STATIC_SCRATCH_BYTES];
 
 namespace {
@@ -107,29 +108,58 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Time split of one long sequence (see the chunk kernel's plans): the number of
-// segments n (0 = none) for H heads and n_chunks chunks. Both passes must fit one
-// wave of the machine (H (2n - 3) CTAs for the state pass, H n for the outputs),
-// and each segment keeps at least MIN_SEG_CHUNKS chunks; the split pays off from
-// n = 3 (two passes over n segments each: n / 2 of the single-pass time).
+// Time split of one long sequence (see the chunk kernel's plans). A split into n
+// segments runs H (2n - 3) CTAs in the state pass (n - 2 transition chains M_j,
+// n - 2 chains R_j and segment 0's output pass per head) and H (n - 1) in the
+// output pass, each over about n_chunks / n chunks, so a call costs about
+// 2 / n of the single pass when both passes fit one wave of SMs. The output pass
+// must fit one wave. The transition chains come first in the state pass and stop
+// as soon as their state is exactly zero; for segments of SPLIT_EARLY_CHUNKS
+// chunks or more the plan counts on that (the erase and the decay shrink every
+// direction of the state: with unit keys and beta near 0.5 the transition loses
+// about e^-0.2 per chunk even without decay, so it underflows to zero within a
+// few hundred chunks), and otherwise plans for the pass taking as many waves as
+// it has CTAs for. Every segment keeps at least MIN_SEG_CHUNKS chunks, and the
+// plan's scratch must fit the bytes available.
 constexpr int MIN_SEG_CHUNKS = 16;
 constexpr int MAX_SEGMENTS = 64;
+constexpr int64_t SPLIT_EARLY_CHUNKS = 512;
 
-int segment_count(int32_t n_heads, int64_t n_chunks) {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return 0;
+size_t segment_workspace_bytes(int n_seg, int32_t n_heads) {
+  return n_seg >= 3 ? (size_t)kda::seg::slots(n_seg) * n_heads * kda::D * kda::D * sizeof(float) : 0;
+}
+
+int split_segments(int32_t n_heads, int64_t n_chunks, int sms, size_t max_bytes) {
   int best = 0;
+  double best_cost = 1.0;   // the single pass, in units of its own time
   for (int n = 3; n <= MAX_SEGMENTS; ++n) {
-    if ((int64_t)n_heads * (2 * n - 3) > sms || n_chunks < (int64_t)n * MIN_SEG_CHUNKS) break;
-    best = n;
+    if (n_chunks < (int64_t)n * MIN_SEG_CHUNKS) break;
+    if ((int64_t)n_heads * (n - 1) > sms) break;
+    if (segment_workspace_bytes(n, n_heads) > max_bytes) break;
+    const double seg = 1.0 / n;
+    const int64_t ctas1 = (int64_t)n_heads * (2 * n - 3);
+    double pass1;
+    if (ctas1 <= sms)
+      pass1 = seg;
+    else if (n_chunks / n >= SPLIT_EARLY_CHUNKS)
+      pass1 = 1.05 * seg;
+    else
+      pass1 = seg * (double)((ctas1 + sms - 1) / sms);
+    const double cost = pass1 + seg;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = n;
+    }
   }
   return best;
 }
 
-size_t segment_workspace_bytes(int n_seg, int32_t n_heads) {
-  return n_seg >= 3 ? (size_t)kda::seg::slots(n_seg) * n_heads * kda::D * kda::D * sizeof(float) : 0;
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return sms;
 }
 
 // Packed batches: a launch order by decreasing length (one int32 per sequence),
@@ -181,7 +211,8 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.t_total = t_total;
   a.plan = PLAN_SEQ;
   a.n_seg = 0;
-  a.seg_chunks = 0;
+  a.seg_base = 0;
+  a.seg_rem = 0;
   a.seg_states = nullptr;
   a.seq_order = nullptr;
   if (seq_order != nullptr && cu_seqlens != nullptr && n_seqs > 1) {
@@ -196,27 +227,26 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
     kda_chunk_tc_kernel<false><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
     return launch_status();
   }
-  // time split: segment states, the scan over segments, then the outputs
+  // time split: segment states (with segment 0's output), the scan over segments,
+  // then the outputs of segments 1 .. n-1
   const int64_t n_chunks = (t_total + kda::CHUNK - 1) / kda::CHUNK;
   a.n_seg = n_seg;
-  a.seg_chunks = (int)((n_chunks + n_seg - 1) / n_seg);
+  a.seg_base = (int)(n_chunks / n_seg);
+  a.seg_rem = (int)(n_chunks % n_seg);
   a.seg_states = seg_states;
   a.plan = PLAN_STATES;
-  // (the state pass writes no output: the lean instantiation)
   kda_chunk_tc_kernel<true><<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
-  if (n_seg > 2) {
-    if (cudaFuncSetAttribute(kda::seg::kda_segment_scan_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kda::seg::SCAN_SMEM) != cudaSuccess)
-      return KDA_ERR_CUDA;
-    kda::seg::kda_segment_scan_kernel<<<(unsigned)n_heads, kda::seg::SCAN_THREADS,
-                                         kda::seg::SCAN_SMEM, stream>>>(seg_states, n_heads, n_seg);
-    if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
-  }
+  if (cudaFuncSetAttribute(kda::seg::kda_segment_scan_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kda::seg::SCAN_SMEM) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  kda::seg::kda_segment_scan_kernel<<<(unsigned)n_heads, kda::seg::SCAN_THREADS, kda::seg::SCAN_SMEM,
+                                       stream>>>(seg_states, n_heads, n_seg);
+  if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
   a.plan = PLAN_OUTPUTS;
-  kda_chunk_tc_kernel<false><<<(unsigned)(n_heads * n_seg), THREADS, SMEM_BYTES, stream>>>(
+  kda_chunk_tc_kernel<false><<<(unsigned)(n_heads * (n_seg - 1)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   return launch_status();
 }
@@ -230,11 +260,12 @@ bool use_tc(const int32_t* cu_seqlens, int32_t n_seqs, int64_t t_total, int32_t 
   return qkv_dtype == KDA_BF16 && t_total >= kda::CHUNK &&
          t_total < (int64_t)INT32_MAX - 4 * kda::CHUNK && (int64_t)n_seqs * n_heads < (int64_t)INT32_MAX;
 }
+// Segments of the time split for a call with max_bytes of scratch (0: no split).
 int plan_segments(const int32_t* cu_seqlens, int32_t n_seqs, int64_t t_total, int32_t n_heads,
-                  kda_dtype qkv_dtype) {
+                  kda_dtype qkv_dtype, size_t max_bytes) {
   if (!use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype) || cu_seqlens != nullptr || n_seqs != 1)
     return 0;
-  return segment_count(n_heads, (t_total + kda::CHUNK - 1) / kda::CHUNK);
+  return split_segments(n_heads, (t_total + kda::CHUNK - 1) / kda::CHUNK, device_sms(), max_bytes);
 }
 
 template <typename TQ, typename TG>
@@ -260,23 +291,45 @@ int launch_decode_tokens(const void* q, const void* k, const void* v, const void
 }
 static_assert(KDA_DECODE_MAX_TOKENS == kda::DEC_MAX_TOKENS, "token limit of the ABI and the kernel");
 
-// Device address of g_kda_static_scratch on the current device. In host code the
+// Device address of g_kda_static_scratch in the current context. In host code the
 // array's name only stands in for the symbol, so the address is looked up once per
-// device, with that device current, and kept.
+// device, with that device current, and kept together with the context it belongs
+// to: a new context on the same device (after cudaDeviceReset, say) looks it up again.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
 constexpr int MAX_STATIC_DEVICES = 64;
 std::mutex g_static_mu;
 void* g_static_addr[MAX_STATIC_DEVICES] = {};
+CUcontext g_static_ctx[MAX_STATIC_DEVICES] = {};
 
 int static_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_STATIC_DEVICES)
     return KDA_ERR_CUDA;
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  CUcontext ctx = nullptr;
+  if (get_ctx == nullptr || get_ctx(&ctx) != CUDA_SUCCESS) return KDA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (g_static_addr[dev] == nullptr) {
+  if (ctx == nullptr || g_static_addr[dev] == nullptr || g_static_ctx[dev] != ctx) {
+    // (the look-up makes the device's primary context current if none was)
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_kda_static_scratch) != cudaSuccess || p == nullptr)
       return KDA_ERR_CUDA;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return KDA_ERR_CUDA;
     g_static_addr[dev] = p;
+    g_static_ctx[dev] = ctx;
   }
   *out = g_static_addr[dev];
   return KDA_OK;
@@ -310,12 +363,28 @@ size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_h
   if (n_heads <= 0 || n_seqs <= 0 || t_total < 0) return 0;
   static const int32_t dummy = 0;
   const int n_seg = plan_segments(has_cu_seqlens ? &dummy : nullptr, n_seqs, t_total, n_heads,
-                                  qkv_dtype);
+                                  qkv_dtype, SIZE_MAX);
   if (n_seg >= 3) return segment_workspace_bytes(n_seg, n_heads);
   if (has_cu_seqlens && n_seqs > 1 &&
       use_tc(&dummy, n_seqs, t_total, n_heads, qkv_dtype))
     return order_workspace_bytes(n_seqs, n_heads);
   return 0;
+}
+
+int kda_chunk_fwd_split_plan(int32_t n_heads, int64_t t_total, int32_t n_sms,
+                             size_t workspace_bytes, int64_t* seg_bounds) {
+  if (n_heads <= 0 || t_total < 0) return KDA_ERR_SHAPE;
+  if (n_sms <= 0) n_sms = device_sms();
+  if (n_sms <= 0) return KDA_ERR_CUDA;
+  if (!use_tc(nullptr, 1, t_total, n_heads, KDA_BF16)) return 0;
+  const int64_t n_chunks = (t_total + kda::CHUNK - 1) / kda::CHUNK;
+  const int n_seg = split_segments(n_heads, n_chunks, n_sms, workspace_bytes);
+  if (n_seg >= 3 && seg_bounds != nullptr) {
+    const int base = (int)(n_chunks / n_seg), rem = (int)(n_chunks % n_seg);
+    for (int j = 0; j < n_seg; ++j) seg_bounds[j] = kda::seg::seg_first_chunk(j, base, rem) * kda::CHUNK;
+    seg_bounds[n_seg] = t_total;
+  }
+  return n_seg;
 }
 
 int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* log_alpha,
@@ -327,8 +396,8 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
   if (st != KDA_OK) return st;
   if (workspace && !aligned16(workspace)) return KDA_ERR_ALIGN;
   if (use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype)) {
-    int n_seg = plan_segments(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype);
-    if (workspace == nullptr || workspace_bytes < segment_workspace_bytes(n_seg, n_heads)) n_seg = 0;
+    const int n_seg = workspace == nullptr ? 0 : plan_segments(cu_seqlens, n_seqs, t_total, n_heads,
+                                                               qkv_dtype, workspace_bytes);
     int32_t* order = nullptr;
     const size_t ob = order_workspace_bytes(n_seqs, n_heads);
     if (n_seg == 0 && cu_seqlens != nullptr && workspace != nullptr && ob > 0 && workspace_bytes >= ob)
@@ -347,8 +416,10 @@ int kda_chunk_fwd_static(const void* q, const void* k, const void* v, const floa
   const int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
                                      n_heads, qkv_dtype, o, hT);
   if (st != KDA_OK) return st;
-  if (kda_chunk_fwd_workspace_size(n_seqs, t_total, n_heads, qkv_dtype, cu_seqlens != nullptr) >
-      KDA_STATIC_SCRATCH_BYTES)
+  // (the time split plans within the array; only a packed batch's launch order could
+  // need more than it holds)
+  if (cu_seqlens != nullptr &&
+      kda_chunk_fwd_workspace_size(n_seqs, t_total, n_heads, qkv_dtype, 1) > KDA_STATIC_SCRATCH_BYTES)
     return KDA_ERR_SCRATCH;
   void* scratch = nullptr;
   const int sst = static_scratch_address(&scratch);

@@ -53,6 +53,7 @@
 #pragma once
 
 #include "kda_common.cuh"
+#include "kda_segment.cuh"
 #include "kda_sm100.cuh"
 
 namespace kda {
@@ -145,20 +146,27 @@ enum : int {
 static_assert(NUM_BARS <= NBARS, "barrier slots");
 
 // Work plans. PLAN_SEQ: one CTA per (sequence of cu_seqlens, head). The time split
-// of one long sequence into n_seg segments of seg_chunks chunks (the last takes the
-// rest) runs as PLAN_STATES, then the segment scan, then PLAN_OUTPUTS:
-//   PLAN_STATES (grid H x (2 n_seg - 3)), slot s of head h:
-//     s = 0                 segment 0 from the caller's h0: the state entering segment 1
-//     s = 1 .. n_seg-2      segment s from a zero state (R_s)
-//     s = n_seg-1 .. 2n-4   segment s-(n_seg-2) from the identity with v = 0 (its
-//                           transition M_s: S_end = M_s S_start + R_s)
-//   and each writes its final state to seg_states[s][h]; no output. This pass runs
-//   the lean instantiation (LEAN = true): no q loads, no Rq tile, no P readout, the
-//   state product only for Delta (N=64), no P Delta product; with v = 0 also no U
-//   product (the Delta product starts from zero).
-//   PLAN_OUTPUTS (grid H x n_seg): segment j from its true entering state (the
-//     caller's h0, slot 0, or the scan's result in slot 2 n_seg - 5 + j), writing o,
-//     and the caller's hT for the last segment.
+// of one long sequence cuts it into n_seg segments of whole chunks, balanced to
+// within one chunk (segment j starts at chunk j*seg_base + min(j, seg_rem); the
+// last one ends at t_total), and runs as PLAN_STATES, the segment scan, then
+// PLAN_OUTPUTS. Slots of seg_states [2 n_seg - 3][H][128][128]: slot 0 the state
+// entering segment 1; slot j (1 .. n_seg-2) R_j, the final state of segment j from
+// a zero start, which the scan overwrites with the state entering segment j+1;
+// slot n_seg-2+j the transition M_j of segment j (S_end = M_j S_start + R_j).
+//   PLAN_STATES (grid H x (2 n_seg - 3)), in block order:
+//     M_1 .. M_{n-2}   segment j from the identity with v = 0: its final state is
+//                      M_j. These come first and end early: once the state is
+//                      exactly zero it stays zero, so the CTA stops there.
+//     R_1 .. R_{n-2}   segment j from a zero state
+//     O_0              segment 0 from the caller's h0, writing its output; its
+//                      final state goes to slot 0
+//   The M and R CTAs write no output and run the lean form of every role (a
+//   CTA-uniform flag, not a second kernel: all CTAs run one body of code, so that
+//   SMs sharing instruction caches fetch the same code): no q loads, no Rq tile, no
+//   P readout, the state product only for Delta (N=64), no P Delta product; with
+//   v = 0 also no U product.
+//   PLAN_OUTPUTS (grid H x (n_seg - 1)): segment j = 1 .. n_seg-1 from slot j-1,
+//     writing o, and the caller's hT for the last segment.
 enum : int { PLAN_SEQ = 0, PLAN_STATES = 1, PLAN_OUTPUTS = 2 };
 
 struct Args {
@@ -173,8 +181,8 @@ struct Args {
   int64_t t_total;
   int plan;
   int n_seg;
-  int seg_chunks;
-  float* seg_states;   // [3 n_seg - 5][H][128][128]
+  int seg_base, seg_rem;   // chunks per segment: seg_base, plus one for the first seg_rem
+  float* seg_states;   // [2 n_seg - 3][H][128][128]
   const int32_t* seq_order;   // PLAN_SEQ: sequences longest first (or null: index order)
 };
 
@@ -191,7 +199,20 @@ struct Ctx {
   bool h0_identity;   // entering state = I (transition of a segment)
   bool v_zero;        // v taken as zero (no loads)
   bool write_o;       // store the output
+  bool stop_on_zero;  // a transition chain: stop once the state is exactly zero
+  bool lean;          // no output: the lean form of every role
 };
+
+// Whether a CTA runs the lean form of the roles. RT = false compiles the full form
+// only (every CTA writes output); RT = true reads the CTA's flag.
+template <bool RT>
+__device__ __forceinline__ bool lean_of(const Ctx& x) { return RT && x.lean; }
+
+// Values of the shared abort word: a role that gives up a wait raises ABORT_TIMEOUT
+// (and flags the device error); the state warps of a transition chain raise
+// ABORT_DONE when the state has become exactly zero. Either way every role leaves
+// its loop at its next wait.
+constexpr int ABORT_TIMEOUT = 1, ABORT_DONE = 2;
 
 // Bounded per-thread wait that also gives up when another role aborted. The
 // thread sleeps in the barrier (suspend hint) instead of spinning. (Out of line,
@@ -202,7 +223,7 @@ __device__ __noinline__ bool wait_b_slow(uint64_t* bar, uint32_t parity, volatil
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > WAIT_NS) {
-      *abort_flag = 1;
+      *abort_flag = ABORT_TIMEOUT;
       flag_error(DEVERR_TIMEOUT);
       return false;
     }
@@ -262,7 +283,7 @@ __device__ __forceinline__ uint64_t kdesc128(uint32_t addr) {
 // ============================================================================
 // TMA and MMA issue (each by the first thread of the role that consumes the result)
 // ============================================================================
-template <bool LEAN>
+template <bool RT>
 __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* map_k,
                                          const CUtensorMap* map_q, int c) {
   const int xk = x.h * D;
@@ -270,10 +291,10 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* map_k,
   uint8_t* st = x.sm + OFF_KQ + (c % 3) * KQ_BYTES;
   const uint32_t koff = (c & 1) ? 8192u : 0u, qoff = 8192u - koff;
   uint64_t* full = &x.bars[B_FULL + c % 3];
-  mbar_arrive_expect_tx(full, (LEAN ? 2 : 4) * 8192);
+  mbar_arrive_expect_tx(full, (lean_of<RT>(x) ? 2 : 4) * 8192);
   tma_load_2d(st + koff, map_k, xk, y, full);
   tma_load_2d(st + 16384 + koff, map_k, xk + 64, y, full);
-  if (LEAN) return;   // no output: q is not needed
+  if (lean_of<RT>(x)) return;   // no output: q is not needed
   tma_load_2d(st + qoff, map_q, xk, y, full);
   tma_load_2d(st + 16384 + qoff, map_q, xk + 64, y, full);
 }
@@ -302,13 +323,13 @@ __device__ void drain(const Ctx& x, int bar) {
 }
 
 // [O | Delta]^T (or [Delta | O]^T) += S''^T [stage tile]^T   (M=128, N=128, K=128);
-// the state operand comes from TMEM. Without output (LEAN) only Delta^T += S''^T (-W')^T
+// the state operand comes from TMEM. Without output (lean) only Delta^T += S''^T (-W')^T
 // (N=64); with v = 0 there is no U to accumulate onto.
-template <bool LEAN>
+template <bool RT>
 __device__ __forceinline__ void issue_crit(const Ctx& x, int c) {
   tc_fence_after();
   const uint32_t kq = smem_u32(x.sm) + OFF_KQ + (c % 3) * KQ_BYTES;
-  if (LEAN) {
+  if (lean_of<RT>(x)) {
     const uint32_t kh = kq + ((c & 1) ? 8192u : 0u);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
@@ -332,7 +353,7 @@ __device__ __forceinline__ uint32_t dpair_col(int kk) { return TM_D + (kk < 2 ? 
 
 // S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T (not without output);
 // Delta^T is the A operand, read from TMEM
-template <bool LEAN>
+template <bool RT>
 __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   tc_fence_after();
   const uint32_t sbase = smem_u32(x.sm);
@@ -343,7 +364,7 @@ __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
     umma_bf16_tmem_a(x.tmem + TM_S, x.tmem + dpair_col(kk),
                      make_sdesc(ck + kk * 2048, 8192, 1024, SWZ_128B), IDESC_Z, 1u);
   umma_commit(&x.bars[B_ZDONE]);
-  if (LEAN) {
+  if (lean_of<RT>(x)) {
     umma_commit(&x.bars[B_CKFREE + (c & 1)]);
     return;
   }
@@ -356,9 +377,9 @@ __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   umma_commit(&x.bars[B_CKFREE + (c & 1)]);
 }
 // U^T = V^T (T beta)^T   (M=128 value columns, N=64, K=64); v read as MN-major A
-template <bool LEAN>
+template <bool RT>
 __device__ __forceinline__ void issue_u(const Ctx& x) {
-  if (LEAN && x.v_zero) {   // U = 0: nothing to compute (the Delta product starts from zero)
+  if (lean_of<RT>(x) && x.v_zero) {   // U = 0: nothing to compute (the Delta product starts from zero)
     umma_commit(&x.bars[B_UDONE]);
     return;
   }
@@ -548,7 +569,7 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, i
   return true;
 }
 
-template <bool LEAN>
+template <bool RT>
 __device__ void prep_a_role(const Ctx& x, const Args& p) {
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
@@ -640,7 +661,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
         uint2* kp = reinterpret_cast<uint2*>(kq + koff + kb * 16384 + swz128(r * 128 + cbyte));
         uint2* qp = reinterpret_cast<uint2*>(kq + qoff + kb * 16384 + swz128(r * 128 + cbyte));
         const uint2 kr = valid ? *kp : make_uint2(0u, 0u);
-        const uint2 qv = (valid && !LEAN) ? *qp : make_uint2(0u, 0u);
+        const uint2 qv = (valid && !lean_of<RT>(x)) ? *qp : make_uint2(0u, 0u);
         float e[4], f[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -649,7 +670,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
         }
         const uint32_t e01 = pack_bf16(e[0], e[1]), e23 = pack_bf16(e[2], e[3]);
         *kp = make_uint2(mul_bf16x2(kr.x, e01), mul_bf16x2(kr.y, e23));
-        if (!LEAN)   // Rq only where there is an output
+        if (!lean_of<RT>(x))   // Rq only where there is an output
           *qp = make_uint2(mul_bf16x2(qv.x, e01), mul_bf16x2(qv.y, e23));
         if (ok)
           *reinterpret_cast<uint2*>(ck + kb * 8192 + swz128(r * 128 + cbyte)) =
@@ -735,7 +756,7 @@ __device__ __forceinline__ void blk_store_tb(uint8_t* tt, int a, int b, const fl
   }
 }
 
-template <bool LEAN>
+template <bool RT>
 __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
                             const CUtensorMap* map_la) {
   const int tid = threadIdx.x - PB_WARP0 * 32;
@@ -760,7 +781,7 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
         const uint32_t par = ((cn - 3) / 3) & 1;
         if (block ? !wait_b(x, B_KQFREE + cn % 3, par) : !mbar_test_wait(fb, par)) return;
       }
-      issue_kq<LEAN>(x, map_k, map_q, cn);
+      issue_kq<RT>(x, map_k, map_q, cn);
       if (cn + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
       ++kq_issued;
     }
@@ -809,7 +830,7 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
             o4.w = (col0 + m + 3 < r) ? br * v[m + 3] : 0.f;
             *reinterpret_cast<float4*>(&aw[r * AW + col0 + m]) = o4;
           }
-        } else if (!LEAN) {   // (P only where there is an output)
+        } else if (!lean_of<RT>(x)) {   // (P only where there is an output)
           uint8_t* pt = ck + 16384;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -1010,7 +1031,7 @@ __device__ __noinline__ void st_store_ragged(uint32_t lane_addr, __nv_bfloat16* 
 // state warps (12-19): the sequential pass over chunks. Thread = (TMEM lane j =
 // value column, half hh of the key channels / of the chunk rows).
 // ============================================================================
-template <bool LEAN>
+template <bool RT>
 __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v,
                            const CUtensorMap* map_o) {
   const int tid = threadIdx.x - ST_WARP0 * 32;
@@ -1025,7 +1046,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 
   // ---- prologue: the fp32 state (h0, identity or zeros) and cleared output accumulators
   st_load_state(x.tmem + TM_S + lb, x.h0, x.h0_identity, j, 64 * hh);
-  if (!LEAN) {
+  if (!lean_of<RT>(x)) {
     tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
     tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
     tmem_st_wait();
@@ -1036,16 +1057,23 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     fence_proxy_async_smem();
   }
 
-  // decay the state over chunk cc in place and write the bf16 operand S''
-  auto s_pass = [&](int cc) {
+  // decay the state over chunk cc in place and write the bf16 operand S''; returns
+  // whether any of this thread's state entries was nonzero (only computed for a
+  // transition chain, which stops once its state is exactly zero)
+  auto s_pass = [&](int cc) -> bool {
     const float* ms = scal_all + (cc % 3) * 256;
     const bool ex = xflag[cc % 3] != 0;
+    uint32_t nz = 0u;
 #pragma unroll 1
     for (int part = 0; part < 2; ++part) {
       const int cb0 = 64 * hh + 32 * part;
       float v[32];
       tmem_ld32(x.tmem + TM_S + lb + cb0, v);
       tmem_ld_wait();
+      if (RT && x.stop_on_zero) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) nz |= __float_as_uint(v[i]) & 0x7FFFFFFFu;
+      }
       uint32_t pk[16];
       if (ex) {   // exact path: the operand is the undecayed state
 #pragma unroll
@@ -1065,6 +1093,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     }
     tmem_st_wait();
     tc_fence_before();
+    return nz != 0u;
   };
 
   // Thread 0 issues this group's tensor-core products and the v loads. Per chunk:
@@ -1096,7 +1125,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       return true;   // not ready yet: issued later, before the chunk's [O | Delta] product
     }
     v_landed = cu + 1;
-    issue_u<LEAN>(x);
+    issue_u<RT>(x);
     u_issued = cu + 1;
     return true;
   };
@@ -1121,118 +1150,127 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   };
 
   bool alive = true;
-  if (n > 0) {
-    if (issuer) {
-      issue_v(x, map_v, 0);
-      v_issued = 1;
-    }
-    alive = wait_b(x, B_TILES + 0, 0);
-    if (alive) s_pass(0);
-    if (issuer && alive) alive = issue_w_of(0, true);
-    alive = alive && w_readout(0);
-    named_bar_sync(BAR_ST, ST_THREADS);
-    if (issuer && alive) {
-      alive = issue_u_of(0, true);
-      if (alive) issue_crit<LEAN>(x, 0);
-    }
+  bool stopped = false;   // a transition chain that stopped early (state exactly zero)
+  if (issuer && n > 0) {
+    issue_v(x, map_v, 0);
+    v_issued = 1;
   }
-  for (int c = 0; c < n; ++c) {
-    const int64_t t0 = x.bos + (int64_t)c * CHUNK;
-    const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
-    // ---- Delta^T fp32 (TMEM, chunk rows 32hh..32hh+31 of lane j) -> bf16 pairs in the
-    //      same lanes, inside the columns just read: the A operand of the update
-    alive = alive && wait_b(x, B_CRIT, c & 1);
-    if (alive) {
-      tc_fence_after();
-      float v[32];
-      tmem_ld32(x.tmem + TM_D + lb + 32 * hh, v);
-      tmem_ld_wait();
-      uint32_t pk[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
-      tmem_st16(x.tmem + TM_D + lb + 48 * hh, pk);
-      tmem_st_wait();
-      tc_fence_before();
-      if (issuer && c + 1 < n) {   // U(c) is done: v of the next chunk may land
-        issue_v(x, map_v, c + 1);
-        v_issued = c + 2;
-      }
-    }
-    // (the output tile of the previous chunk must have been read by its store before
-    //  anyone stages this chunk's output in it: every warp passes this barrier first)
-    if (issuer && c > 0) bulk_wait_read_all();
-    named_bar_sync(BAR_ST, ST_THREADS);
-    if (issuer && alive) {
-      issue_update<LEAN>(x, c);
-      if (c + 1 < n) {
-        alive = issue_w_of(c + 1, false);
-        if (alive && w_issued == c + 2) alive = issue_u_of(c + 1, false);
-      }
-    }
-    // ---- next chunk's decayed state, as soon as this chunk's update has landed
-    if (c + 1 < n) {
-      alive = alive && wait_b(x, B_ZDONE, c & 1) &&
-              wait_b(x, B_TILES + ((c + 1) & 1), ((c + 1) >> 1) & 1);
+  // One pass of the loop per chunk c, plus one to finish the last output. Each step
+  // appears once in the code: the roles' code shares the SM's instruction caches.
+  //   (a) chunk c's decayed state S'' (once the update of chunk c-1 has landed), its
+  //       -W' tile and the [O | Delta] product;
+  //   (b) the output of chunk c-1, off the sequential path;
+  //   (c) Delta of chunk c back into TMEM as bf16 pairs, then the state update.
+  for (int c = 0; c <= n; ++c) {
+    if (c < n) {
+      alive = alive && (c == 0 || wait_b(x, B_ZDONE, (c - 1) & 1)) &&
+              wait_b(x, B_TILES + (c & 1), (c >> 1) & 1);
+      bool nonzero = true;
       if (alive) {
         tc_fence_after();
-        s_pass(c + 1);
+        nonzero = s_pass(c);
       }
-      if (issuer && alive && w_issued < c + 2) alive = issue_w_of(c + 1, true);
-      alive = alive && w_readout(c + 1);
+      if (issuer && alive && w_issued < c + 1) alive = issue_w_of(c, true);
+      alive = alive && w_readout(c);
+      // (the output tile's last store must have read it before (b) stages the next)
+      if (issuer && c > 1) bulk_wait_read_all();
+      if (RT && x.stop_on_zero && c > 0) {
+        // A transition chain whose state is exactly zero after chunk c-1 stays zero
+        // (v = 0, so every later Delta and update is zero too): its final state is
+        // known, and the CTA stops here. The other roles see ABORT_DONE at their
+        // next wait and leave; the update of chunk c-1 has landed.
+        if (!named_bar_or(BAR_ST, ST_THREADS, nonzero || !alive)) {
+          if (tid == 0) *x.abort_flag = ABORT_DONE;
+          stopped = true;
+          break;
+        }
+      } else {
+        named_bar_sync(BAR_ST, ST_THREADS);
+      }
+      if (issuer && alive) {
+        if (u_issued < c + 1) alive = issue_u_of(c, true);
+        if (alive) issue_crit<RT>(x, c);
+      }
+    }
+    if (c > 0 && !lean_of<RT>(x)) {
+      const int co = c - 1;
+      const int64_t t0 = x.bos + (int64_t)co * CHUNK;
+      const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
+      alive = alive && wait_b(x, B_PD, co & 1);
+      if (alive) {
+        tc_fence_after();
+        const uint32_t ro = (co & 1) ? TM_OA : TM_OB;
+        if (L == CHUNK) {
+          // full chunk: into the output tile (its previous store has read it), then one
+          // TMA store of [64 rows][128 columns]
+          float v[32];
+          tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
+          tmem_ld_wait();
+          uint8_t* ot = dt + (j >> 6) * 8192;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            *reinterpret_cast<__nv_bfloat16*>(ot + swz128((32 * hh + i) * 128 + (j & 63) * 2)) =
+                __float2bfloat16_rn(v[i]);
+          fence_proxy_async_smem();
+        } else {
+          // ragged last chunk of a sequence: direct stores of the valid rows only
+          st_store_ragged(x.tmem + ro + lb + 32 * hh, p.o + (size_t)t0 * x.rs + x.h * D + j, x.rs,
+                          32 * hh, L);
+        }
+        tmem_st32_zero(x.tmem + ro + lb + 32 * hh);
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      if (L == CHUNK) {
+        // the warps that do not issue only report their part staged and go on; the
+        // issuing warp waits for all parts and sends the tile
+        if (sw != 0) {
+          named_bar_arrive(BAR_OUT, ST_THREADS);
+        } else {
+          named_bar_sync(BAR_OUT, ST_THREADS);
+          if (issuer && alive) {
+            tma_store_2d(map_o, dt, x.h * D, (int)t0);
+            tma_store_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);
+            bulk_commit_group();
+          }
+        }
+      }
+    }
+    if (c < n) {
+      // ---- Delta^T fp32 (TMEM, chunk rows 32hh..32hh+31 of lane j) -> bf16 pairs in the
+      //      same lanes, inside the columns just read: the A operand of the update
+      alive = alive && wait_b(x, B_CRIT, c & 1);
+      if (alive) {
+        tc_fence_after();
+        float v[32];
+        tmem_ld32(x.tmem + TM_D + lb + 32 * hh, v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+        tmem_st16(x.tmem + TM_D + lb + 48 * hh, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        if (issuer && c + 1 < n) {   // U(c) is done: v of the next chunk may land
+          issue_v(x, map_v, c + 1);
+          v_issued = c + 2;
+        }
+      }
       named_bar_sync(BAR_ST, ST_THREADS);
       if (issuer && alive) {
-        if (u_issued < c + 2) alive = issue_u_of(c + 1, true);
-        if (alive) issue_crit<LEAN>(x, c + 1);
-      }
-    }
-    // ---- output of chunk c (off the sequential path), then clear its columns
-    if (LEAN) continue;
-    alive = alive && wait_b(x, B_PD, c & 1);
-    if (alive) {
-      tc_fence_after();
-      const uint32_t ro = (c & 1) ? TM_OA : TM_OB;
-      if (!x.write_o) {
-        // (segment state pass: no output)
-      } else if (L == CHUNK) {
-        // full chunk: into the output tile (its previous store has read it), then one
-        // TMA store of [64 rows][128 columns]
-        float v[32];
-        tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
-        tmem_ld_wait();
-        uint8_t* ot = dt + (j >> 6) * 8192;
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          *reinterpret_cast<__nv_bfloat16*>(ot + swz128((32 * hh + i) * 128 + (j & 63) * 2)) =
-              __float2bfloat16_rn(v[i]);
-        fence_proxy_async_smem();
-      } else {
-        // ragged last chunk of a sequence: direct stores of the valid rows only
-        st_store_ragged(x.tmem + ro + lb + 32 * hh, p.o + (size_t)t0 * x.rs + x.h * D + j, x.rs,
-                        32 * hh, L);
-      }
-      tmem_st32_zero(x.tmem + ro + lb + 32 * hh);
-      tmem_st_wait();
-      tc_fence_before();
-    }
-    if (L == CHUNK && x.write_o) {
-      // the warps that do not issue only report their part staged and move on to the
-      // next chunk; the issuing warp waits for all parts and sends the tile
-      if (sw != 0) {
-        named_bar_arrive(BAR_OUT, ST_THREADS);
-        continue;
-      }
-      named_bar_sync(BAR_OUT, ST_THREADS);
-      if (issuer && alive) {
-        tma_store_2d(map_o, dt, x.h * D, (int)t0);
-        tma_store_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);
-        bulk_commit_group();
+        issue_update<RT>(x, c);
+        if (c + 1 < n) {
+          alive = issue_w_of(c + 1, false);
+          if (alive && w_issued == c + 2) alive = issue_u_of(c + 1, false);
+        }
       }
     }
   }
-  // ---- final state
-  if (n > 0) alive = alive && wait_b(x, B_ZDONE, (n - 1) & 1);
+  // ---- final state (after an early stop: the zero state, whose last update has landed)
+  if (n > 0 && !stopped) alive = alive && wait_b(x, B_ZDONE, (n - 1) & 1);
   tc_fence_after();
-  if (x.hT && alive && !*x.abort_flag) st_store_state(x.tmem + TM_S + lb, x.hT, j, 64 * hh);
+  if (x.hT && alive && *x.abort_flag != ABORT_TIMEOUT)
+    st_store_state(x.tmem + TM_S + lb, x.hT, j, 64 * hh);
   if (issuer) {
     bulk_wait_all();
     drain(x, B_FIN_C);
@@ -1241,9 +1279,13 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 }
 
 // ============================================================================
-// kernel: one CTA per (sequence, head)
+// kernel: one CTA per (sequence, head), or per (segment, head) of a time split.
+// RT = false (PLAN_SEQ, PLAN_OUTPUTS): every CTA writes output, and only the full
+// form of the roles is compiled. RT = true (PLAN_STATES): each CTA's flag picks the
+// lean or the full form at run time, in one body of code, so that the SMs of a TPC,
+// which share instruction caches, fetch the same code whichever CTAs they hold.
 // ============================================================================
-template <bool LEAN>
+template <bool RT>
 __global__ void __launch_bounds__(THREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_la,
@@ -1262,6 +1304,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.h0_identity = false;
   x.v_zero = false;
   x.write_o = true;
+  x.stop_on_zero = false;
+  x.lean = false;
   const size_t state_elems = (size_t)D * D;
   if (args.plan == PLAN_SEQ) {
     // CTAs start in index order; with seq_order the longest sequences go first, so
@@ -1277,31 +1321,40 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
     x.hT = args.hT ? args.hT + sidx : nullptr;
   } else {
     const int ns = args.n_seg;
+    auto state_slot = [&](int s) { return args.seg_states + ((size_t)s * H + x.h) * state_elems; };
     int seg;
     if (args.plan == PLAN_STATES) {
-      x.write_o = false;
-      x.h0 = nullptr;
-      if (slot == 0) {
-        seg = 0;
-        x.h0 = args.h0 ? args.h0 + (size_t)x.h * state_elems : nullptr;
-      } else if (slot <= ns - 2) {
-        seg = slot;
-      } else {
-        seg = slot - (ns - 2);
+      if (slot < ns - 2) {              // M_j, j = slot + 1
+        seg = slot + 1;
+        x.lean = true;
+        x.write_o = false;
+        x.h0 = nullptr;
         x.h0_identity = true;
         x.v_zero = true;
-      }
-      x.hT = args.seg_states + ((size_t)slot * H + x.h) * state_elems;
-    } else {
-      seg = slot;
-      if (seg == 0)
+        x.stop_on_zero = true;
+        x.hT = state_slot(ns - 2 + seg);
+      } else if (slot < 2 * ns - 4) {   // R_j, j = slot - (n - 3)
+        seg = slot - (ns - 3);
+        x.lean = true;
+        x.write_o = false;
+        x.h0 = nullptr;
+        x.hT = state_slot(seg);
+      } else {                          // O_0
+        seg = 0;
         x.h0 = args.h0 ? args.h0 + (size_t)x.h * state_elems : nullptr;
-      else
-        x.h0 = args.seg_states + ((size_t)(seg == 1 ? 0 : 2 * ns - 5 + seg) * H + x.h) * state_elems;
+        x.hT = state_slot(0);
+      }
+    } else {
+      seg = slot + 1;
+      x.h0 = state_slot(seg - 1);
       x.hT = (seg == ns - 1 && args.hT) ? args.hT + (size_t)x.h * state_elems : nullptr;
     }
-    x.bos = (int64_t)seg * args.seg_chunks * CHUNK;
-    x.eos = (seg == ns - 1) ? args.t_total : x.bos + (int64_t)args.seg_chunks * CHUNK;
+    auto seg_start = [&](int j) { return seg::seg_first_chunk(j, args.seg_base, args.seg_rem) * CHUNK; };
+    x.bos = seg_start(seg);
+    x.eos = (seg == ns - 1) ? args.t_total : seg_start(seg + 1);
+    if (x.bos > args.t_total) x.bos = args.t_total;
+    if (x.eos > args.t_total) x.eos = args.t_total;
+    if (x.eos < x.bos) x.eos = x.bos;
   }
   x.n_chunks = (int)((x.eos - x.bos + CHUNK - 1) / CHUNK);
 
@@ -1329,11 +1382,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.tmem = *tmem_slot;
 
   if (warp < PA_WARPS) {
-    prep_a_role<LEAN>(x, args);
+    prep_a_role<RT>(x, args);
   } else if (warp < ST_WARP0) {
-    prep_b_role<LEAN>(x, &map_k, &map_q, &map_la);
+    prep_b_role<RT>(x, &map_k, &map_q, &map_la);
   } else {
-    state_role<LEAN>(x, args, &map_v, &map_o);
+    state_role<RT>(x, args, &map_v, &map_o);
   }
   tc_fence_before();
   __syncthreads();

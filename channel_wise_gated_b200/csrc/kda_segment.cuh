@@ -3,13 +3,13 @@
 // Every step of the recurrence (Kimi Linear summary, section 3) is affine in the
 // state, so a segment of chunks maps its entering state S to M S + R, with M the
 // product of its per-token transitions (I - beta k k^T) Diag(alpha) and R its final
-// state from a zero start. The chunk kernel's state pass computes, per head, the
-// exact state entering segment 1 (slot 0), R_s (slots 1 .. n-2) and M_s (slots
-// n-1 .. 2n-4, the final state from the identity with v = 0). This kernel then
-// walks the segments in order,
-//     S_j = M_{j-1} S_{j-1} + R_{j-1},   j = 2 .. n-1,
-// writing S_j to slot 2n-5+j, all in fp32. One CTA per head; n-2 products of
-// 128 x 128 matrices, a few microseconds in all.
+// state from a zero start. The chunk kernel's state pass leaves, per head, the
+// exact state entering segment 1 in slot 0, R_j in slot j and M_j in slot n-2+j
+// (j = 1 .. n-2; M_j is the final state from the identity with v = 0). This kernel
+// then walks the segments in order,
+//     S_{j+1} = M_j S_j + R_j,   j = 1 .. n-2   (S_1 = slot 0),
+// writing S_{j+1} over R_j in slot j, all in fp32. One CTA per head; n-2 products
+// of 128 x 128 matrices, a few microseconds in all.
 #pragma once
 
 #include "kda_common.cuh"
@@ -22,23 +22,30 @@ constexpr int SP = D + 4;   // smem pitch of the row-major copies (keeps float4 
 constexpr size_t SCAN_SMEM = 2 * (size_t)D * SP * sizeof(float);
 
 // Slots of the segment-state buffer [slots][H][128][128] (see the chunk kernel's plans).
-__host__ __device__ constexpr int slots(int n_seg) { return 3 * n_seg - 5; }
+__host__ __device__ constexpr int slots(int n_seg) { return 2 * n_seg - 3; }
+
+// First chunk of segment j when n_chunks chunks are cut into n_seg segments balanced
+// to within one chunk: seg_base = n_chunks / n_seg, seg_rem = n_chunks % n_seg, and
+// the first seg_rem segments take one chunk more. Segment j covers chunks
+// [seg_first_chunk(j), seg_first_chunk(j + 1)); seg_first_chunk(n_seg) = n_chunks.
+__host__ __device__ inline int64_t seg_first_chunk(int j, int seg_base, int seg_rem) {
+  return (int64_t)j * seg_base + (j < seg_rem ? j : seg_rem);
+}
 
 __global__ void __launch_bounds__(SCAN_THREADS)
 kda_segment_scan_kernel(float* __restrict__ states, int n_heads, int n_seg) {
   extern __shared__ __align__(16) float sm[];
-  float* Ms = sm;             // M_{j-1}, row-major, pitch SP
-  float* Ss = sm + D * SP;    // S_{j-1}
+  float* Ms = sm;             // M_j, row-major, pitch SP
+  float* Ss = sm + D * SP;    // S_j
   const int h = blockIdx.x, tid = threadIdx.x;
   const size_t E = (size_t)D * D;
   auto slot = [&](int s) { return states + ((size_t)s * n_heads + h) * E; };
   // thread tile: rows r0..r0+7, columns c0..c0+7 of the 128 x 128 result
   const int r0 = 8 * (tid >> 4), c0 = 8 * (tid & 15);
-  for (int j = 2; j < n_seg; ++j) {
-    const float* M = slot(n_seg - 3 + j);                    // M_{j-1}
-    const float* S = slot(j == 2 ? 0 : 2 * n_seg - 6 + j);   // S_{j-1}
-    const float* R = slot(j - 1);                            // R_{j-1}
-    float* out = slot(2 * n_seg - 5 + j);                    // S_j
+  for (int j = 1; j <= n_seg - 2; ++j) {
+    const float* M = slot(n_seg - 2 + j);       // M_j
+    const float* S = slot(j - 1);               // S_j (slot 0, or the previous result)
+    float* RS = slot(j);                        // R_j in, S_{j+1} out
     for (int i = tid; i < D * D / 4; i += SCAN_THREADS) {
       const int r = (4 * i) / D, c = (4 * i) % D;
       *reinterpret_cast<float4*>(&Ms[r * SP + c]) = reinterpret_cast<const float4*>(M)[i];
@@ -63,12 +70,13 @@ kda_segment_scan_kernel(float* __restrict__ states, int n_heads, int n_seg) {
 #pragma unroll
         for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
     }
+    // each element of R_j is read and overwritten by the same thread
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
         const size_t e = (size_t)(r0 + a) * D + c0 + b;
-        out[e] = acc[a][b] + R[e];
+        RS[e] = acc[a][b] + RS[e];
       }
     __syncthreads();
   }

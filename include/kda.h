@@ -105,18 +105,22 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_
  * Every step of the recurrence is affine in the state, so a run of chunks maps
  * its entering state S to M S + R (M: product of the per-token transitions,
  * R: the final state from a zero start). With the time split the sequence is cut
- * into n segments (n >= 3, chosen so that both passes fit one wave of the GPU):
- * a first pass computes, in parallel, the exact state entering segment 1 and
- * (R_s, M_s) of the middle segments; a scan composes them into the state entering
- * every segment; a second pass runs all segments in parallel from those states
- * and writes o and hT. The result is the same recurrence (exact in real
+ * into n >= 3 segments of whole chunks (balanced to within one chunk). A first
+ * pass computes, in parallel, segment 0's output and final state and (R_j, M_j)
+ * of the middle segments; the M_j runs stop early once their state is exactly
+ * zero, which the erase and the decay bring about within a few hundred chunks on
+ * typical inputs. A scan composes the maps into the state entering every segment,
+ * and a second pass runs segments 1 .. n-1 in parallel from those states and
+ * writes o and hT. n is chosen for the current device's SM count (see
+ * kda_chunk_fwd_split_plan). The result is the same recurrence (exact in real
  * arithmetic; fp32 state throughout, bf16 MMA operands as in kda_chunk_fwd).
  *
  * Arguments: as kda_chunk_fwd, plus
  *   workspace        16-byte aligned device scratch, or NULL
- *   workspace_bytes  its size; the split runs only when it is at least
- *                    kda_chunk_fwd_workspace_size(...) > 0, otherwise the call is
- *                    exactly kda_chunk_fwd (single pass)
+ *   workspace_bytes  its size. The split takes the best plan whose scratch fits
+ *                    ((2n - 3) * n_heads * 64 KiB); with NULL, or too little for
+ *                    any split, the call is exactly kda_chunk_fwd (single pass).
+ *                    kda_chunk_fwd_workspace_size(...) bytes give the best plan.
  * The workspace must stay untouched until the stream has passed the call.
  * Returns KDA_OK or a negative kda_status (KDA_ERR_ALIGN for a misaligned workspace).
  */
@@ -124,6 +128,24 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
                      const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                      int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * kda_chunk_fwd_split_plan - the time split kda_chunk_fwd_ws would use for one bf16
+ * sequence of t_total tokens and n_heads heads, given workspace_bytes of scratch
+ * (SIZE_MAX: as much as it wants), on a GPU with n_sms SMs (0: the current
+ * device's). Host-only arithmetic: it launches nothing and, with n_sms > 0,
+ * touches no device.
+ *
+ * Returns the number of segments n (0: no split, the single pass runs), or a
+ * negative kda_status (KDA_ERR_SHAPE for n_heads <= 0 or t_total < 0,
+ * KDA_ERR_CUDA if n_sms is 0 and the device cannot be queried). If seg_bounds is
+ * not NULL and n >= 3, it receives n + 1 token offsets: segment j covers tokens
+ * [seg_bounds[j], seg_bounds[j+1]), seg_bounds[0] = 0, seg_bounds[n] = t_total,
+ * every inner offset a multiple of 64. At most KDA_MAX_SEGMENTS segments.
+ */
+#define KDA_MAX_SEGMENTS 64
+int kda_chunk_fwd_split_plan(int32_t n_heads, int64_t t_total, int32_t n_sms,
+                             size_t workspace_bytes, int64_t* seg_bounds);
 
 /*
  * kda_chunk_fwd_workspace_size - bytes of workspace kda_chunk_fwd_ws would use for
@@ -148,18 +170,22 @@ size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_h
  *
  * Scratch: one __device__ array of KDA_STATIC_SCRATCH_BYTES (16 MiB), 256-byte
  * aligned, in every GPU context that loads the library, held until the process
- * exits. The time split of one long sequence uses (3n - 5) * n_heads * 64 KiB of
- * it (n segments; at most 13.75 MiB on a 148-SM B200) and a packed batch of more
- * CTAs than SMs uses 4 bytes per sequence.
+ * exits. The time split of one long sequence plans within it ((2n - 3) * n_heads
+ * * 64 KiB for n segments: 14 MiB for 32 heads in 5 segments), so for a few head
+ * counts it splits into fewer segments than kda_chunk_fwd_ws given a workspace of
+ * kda_chunk_fwd_workspace_size(...) bytes would. A packed batch of more CTAs than
+ * SMs uses 4 bytes per sequence.
  *
- * Limit: a call for which kda_chunk_fwd_workspace_size(...) exceeds
- * KDA_STATIC_SCRATCH_BYTES is rejected with KDA_ERR_SCRATCH before anything is
- * launched (on a 148-SM B200 no call reaches it; parts with more SMs can).
+ * Limit: a packed batch whose launch order needs more than KDA_STATIC_SCRATCH_BYTES
+ * is rejected with KDA_ERR_SCRATCH before anything is launched (the order is kept
+ * for at most 16,384 sequences, 64 KiB, so no call reaches it).
  *
- * Set-up: the first call on each device, made with that device current, looks up
- * the array's device address (cudaGetSymbolAddress, which may load this library's
- * kernels onto the device) and keeps it for later calls; make that first call
- * before any stream capture on the device. A failed look-up returns KDA_ERR_CUDA.
+ * Set-up: the first call in each device context, made with that device current,
+ * looks up the array's device address (cudaGetSymbolAddress, which may load this
+ * library's kernels onto the device) and keeps it, with the context, for later
+ * calls; make that first call before any stream capture on the device. A new
+ * context on the device (after cudaDeviceReset, say) looks the address up again.
+ * A failed look-up returns KDA_ERR_CUDA.
  *
  * Sharing: every call on a device, from any stream or host thread, uses the same
  * array and leaves its contents behind. Nothing in it has to start at zero (each
@@ -240,6 +266,12 @@ int kda_decode_tokens(const void* q, const void* k, const void* v, const void* l
  * Synchronises `stream`. Returns KDA_OK, KDA_ERR_SEQLENS (a kernel saw
  * cu_seqlens that were not monotone or ran past t_total, and clamped them),
  * KDA_ERR_TIMEOUT (a kernel gave up a bounded wait), or KDA_ERR_CUDA.
+ *
+ * The error word is one per GPU context and process, not per call or per stream:
+ * every kernel of this library on the device ORs its errors into it, and any
+ * caller's read clears it. A caller that runs the library on several streams
+ * cannot tell from it which call failed, and one stream's read hides an error
+ * from the others; synchronise the streams and read it once where that matters.
  */
 int kda_device_status(cudaStream_t stream);
 

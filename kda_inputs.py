@@ -165,3 +165,29 @@ def make_decode_config(device="cpu", n_seqs=None, steps=None):
     c = DECODE_CONFIG
     return make_decode(n_seqs or c.n_seqs, c.n_heads, steps or c.steps, c.qkv_dtype,
                        c.gate_dtype, c.x_mean, c.state_std, c.seed, device)
+
+
+def make_parallel_keys(T: int, n_heads: int, qkv_dtype=torch.bfloat16, eps: float = 1e-2,
+                       run: int = 16, beta_lo: float = 0.98, x_mean: float = 8.0,
+                       h0_std: float = 1.0, seed: int = 0, device="cpu", d: int = D):
+    """A hard case for the chunk form's triangular solve: one sequence whose keys come
+    in runs of `run` nearly parallel unit vectors (k_t = normalise(k_base + eps * n_t),
+    a new base direction per run), erase strengths beta ~ U[beta_lo, 1], decay close to
+    one (log_alpha = logsigmoid(x), x ~ N(x_mean, 1)) and a large initial state
+    (h0 ~ N(0, h0_std)). q and v are drawn as in make_prefill. Same dict as make_prefill.
+    """
+    g = _gen(device, seed)
+    shp = (T, n_heads, d)
+    q = _unit_rows(torch.randn(shp, generator=g, device=device)).to(qkv_dtype)
+    n_runs = (T + run - 1) // run
+    base = torch.randn((n_runs, n_heads, d), generator=g, device=device)
+    base = base.repeat_interleave(run, dim=0)[:T]
+    k = _unit_rows(_unit_rows(base) + eps * torch.randn(shp, generator=g, device=device))
+    k = k.to(qkv_dtype)
+    v = torch.randn(shp, generator=g, device=device).to(qkv_dtype)
+    x = torch.randn(shp, generator=g, device=device) + x_mean
+    la = torch.nn.functional.logsigmoid(x).float()
+    b = (beta_lo + (1.0 - beta_lo) * torch.rand((T, n_heads), generator=g, device=device)).float()
+    h0_t = (torch.randn((1, n_heads, d, d), generator=g, device=device) * h0_std).float()
+    cu = torch.tensor([0, T], dtype=torch.int32, device=device)
+    return dict(q=q, k=k, v=v, log_alpha=la, beta=b, h0=h0_t, cu_seqlens=cu, lens=[T])

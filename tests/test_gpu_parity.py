@@ -63,12 +63,8 @@ def _run(kda, inp, kernel="auto"):
 
 
 def _split_segments(kda, T, H):
-    """Segments the time split uses for one bf16 sequence (0: no split)."""
-    ws = kda._native.load().kda_chunk_fwd_workspace_size(1, T, H, kda._native.KDA_BF16, 0)
-    if ws == 0:
-        return 0
-    slots = ws // (H * 128 * 128 * 4)
-    return (slots + 5) // 3
+    """Segments the time split uses for one bf16 sequence on this device (0: no split)."""
+    return max(len(kda.split_plan(H, T)) - 1, 0)
 
 
 @pytest.mark.parametrize("kernel", ["auto", "simt"])
@@ -95,10 +91,9 @@ def test_config2_varlen(kda):
     inp = kda_inputs.make_config(2, device="cuda")
     assert len(inp["lens"]) == 16
     o, hT = _run(kda, inp)
-    heads = [0, 13, 31]   # sampled heads, every sequence, every token
-    o_ref, h_ref = _oracle(inp, heads)
-    e_o = rel_err(o[:, heads], o_ref)
-    e_s = rel_err(hT[:, heads], h_ref)
+    o_ref, h_ref = _oracle(inp)   # all 32 heads, every sequence, every token
+    e_o = rel_err(o, o_ref)
+    e_s = rel_err(hT, h_ref)
     print(f"config2: o {e_o:.2e} hT {e_s:.2e}")
     assert e_o <= TOL_BF16 and e_s <= TOL_BF16
     assert kda.device_status() == 0
@@ -351,3 +346,92 @@ def test_bad_seqlens_are_clamped_and_reported(kda):
     kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], cu_seqlens=cu)
     assert kda.device_status() == kda._native.KDA_ERR_SEQLENS
     assert kda.device_status() == 0   # read clears it
+
+
+@pytest.mark.parametrize("eps", [1e-1, 1e-2])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_nearly_parallel_keys_full_erase(kda, eps, dtype):
+    """The triangular solve's hard case: runs of nearly parallel unit keys, erase
+    strength beta in [0.98, 1], decay close to one and a large initial state (std 1),
+    so that I + A is close to singular within a run and T = (I + A)^-1 is far from
+    the identity. bf16 takes the tensor-core kernel (T beta rounded to bf16 as an
+    MMA operand), fp32 the CUDA-core kernel."""
+    T, H = 64 * 6 + 17, 4
+    for run in (16, 64):
+        inp = kda_inputs.make_parallel_keys(T, H, dtype, eps=eps, run=run,
+                                            seed=int(1e4 * eps) + run, device="cuda")
+        o, hT = _run(kda, inp)
+        o_ref, h_ref = _oracle(inp)
+        tol = TOL_F32 if dtype == torch.float32 else TOL_BF16
+        e_o, e_s = rel_err(o, o_ref), rel_err(hT, h_ref)
+        print(f"parallel keys eps={eps} run={run} {dtype}: o {e_o:.2e} hT {e_s:.2e}")
+        assert e_o <= tol and e_s <= tol
+
+
+def test_nearly_parallel_keys_time_split(kda):
+    """The same hard case through the time split (32 heads, 3 segments): the segment
+    transitions barely shrink, and the state enters every segment large."""
+    T, H = 64 * 60 + 9, 32
+    assert _split_segments(kda, T, H) == 3
+    inp = kda_inputs.make_parallel_keys(T, H, torch.bfloat16, eps=1e-2, run=32, seed=77,
+                                        device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    e_o, e_s = rel_err(o, o_ref), rel_err(hT, h_ref)
+    print(f"parallel keys, split: o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+
+
+def test_time_split_uneven_segments_4_heads(kda):
+    """4 heads over 321 chunks: 20 segments whose lengths differ by one chunk (the
+    chunk count is not a multiple of the segment count), plus a ragged tail."""
+    T, H = 321 * 64 + 13, 4
+    bounds = kda.split_plan(H, T)
+    assert len(bounds) - 1 == 20
+    sizes = np.diff(bounds)
+    assert bounds[0] == 0 and bounds[-1] == T and sizes.min() > 15 * 64   # >= 16 chunks
+    assert len(set(sizes[:-1].tolist())) == 2   # 17 and 16 chunks
+    inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 3.0, True, seed=86,
+                                  device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    e_o, e_s = rel_err(o, o_ref), rel_err(hT, h_ref)
+    print(f"4 heads, 20 segments: o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+    o_1, h_1 = _run(kda, inp, kernel="single")
+    assert rel_err(o, o_1.double().cpu().numpy()) <= TOL_BF16
+    assert rel_err(hT, h_1.double().cpu().numpy()) <= TOL_BF16
+
+
+@pytest.mark.parametrize("x_mean", [0.0, -5.0])
+def test_time_split_transitions_vanish(kda, x_mean):
+    """Strong decay (about -50 or -320 nats per chunk): every segment transition M_j
+    becomes exactly zero after a chunk or two, so its CTA stops early while the other
+    roles are still ahead of it. Results must match the oracle and the single pass."""
+    T, H = 64 * 100 + 5, 16
+    assert _split_segments(kda, T, H) == 6
+    inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, x_mean, True, seed=87,
+                                  device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    e_o, e_s = rel_err(o, o_ref), rel_err(hT, h_ref)
+    print(f"transitions vanish (mu {x_mean}): o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= max(TOL_BF16, 1e-30)
+    o_1, h_1 = _run(kda, inp, kernel="single")
+    assert rel_err(o, o_1.double().cpu().numpy()) <= TOL_BF16
+
+
+def test_time_split_five_segments_long(kda):
+    """32 heads over 3000 chunks: 5 segments of 600 chunks, with the transition runs
+    expected to end early (the headline plan at a fifth of its length). The oracle
+    follows 3 heads end to end."""
+    T, H = 3000 * 64, 32
+    assert _split_segments(kda, T, H) == 5
+    inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 4.0, True, seed=88,
+                                  device="cuda")
+    o, hT = _run(kda, inp)
+    heads = [0, 17, 31]
+    o_ref, h_ref = _oracle(inp, heads)
+    e_o, e_s = rel_err(o[:, heads], o_ref), rel_err(hT[:, heads], h_ref)
+    print(f"5 segments: o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16

@@ -1,0 +1,98 @@
+"""Host-side arithmetic of the time split (kda_chunk_fwd_split_plan), on the CPU.
+
+The plan decides how one long bf16 sequence is cut into segments, and the kernels
+read exactly the token ranges it implies. These checks run without a GPU: the
+planning call with an explicit SM count touches no device.
+
+For every head count from 1 to 148 on a 148-SM part, and chunk counts around every
+multiple of the segment counts, a plan must
+  * cover the sequence exactly: bounds start at 0, end at t_total, strictly increase,
+    and every inner bound is a whole chunk;
+  * give every segment at least 16 chunks, with lengths differing by at most one chunk
+    (the last segment alone may end in a partial chunk);
+  * fit one wave of SMs with its output pass: H (n - 1) <= SMs;
+  * fit the scratch it is given: (2n - 3) * H * 64 KiB.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+
+from channel_wise_gated_b200 import _native
+
+SMS = 148
+SLOT = 128 * 128 * 4
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from channel_wise_gated_b200 import build
+    build.build()
+    return _native.load()
+
+
+def _plan(lib, H, T, sms=SMS, ws=_native.SIZE_MAX):
+    b = (ctypes.c_int64 * (_native.KDA_MAX_SEGMENTS + 1))()
+    n = lib.kda_chunk_fwd_split_plan(H, T, sms, ws, b)
+    return n, [int(b[i]) for i in range(n + 1)] if n >= 3 else []
+
+
+def _check(H, T, n, bounds, sms, ws):
+    if n == 0:
+        return
+    assert 3 <= n <= _native.KDA_MAX_SEGMENTS
+    assert H * (n - 1) <= sms
+    assert (2 * n - 3) * H * SLOT <= ws
+    assert bounds[0] == 0 and bounds[-1] == T
+    b = np.array(bounds)
+    assert np.all(np.diff(b) > 0)
+    assert np.all(b[:-1] % 64 == 0)
+    chunks = np.diff(np.append(b[:-1] // 64, (T + 63) // 64))
+    assert chunks.min() >= 16
+    assert chunks.max() - chunks.min() <= 1
+
+
+@pytest.mark.parametrize("H", list(range(1, SMS + 1)))
+def test_plan_covers_sequence(lib, H):
+    seen = set()
+    for n_chunks in list(range(16, 400, 7)) + [512, 1000, 1024, 3000, 16384]:
+        for tail in (0, 1, 63):
+            T = n_chunks * 64 - (64 - tail if tail else 0)
+            n, bounds = _plan(lib, H, T)
+            assert n >= 0
+            _check(H, T, n, bounds, SMS, _native.SIZE_MAX)
+            seen.add(n)
+    if H <= SMS // 2:
+        assert max(seen) >= 3   # some length splits
+
+
+def test_reported_case_4_heads_321_chunks(lib):
+    # 4 heads and 321 chunks: 20 segments of 17 and 16 chunks (no segment past the end)
+    n, bounds = _plan(lib, 4, 321 * 64)
+    assert n == 20
+    _check(4, 321 * 64, n, bounds, SMS, _native.SIZE_MAX)
+
+
+def test_headline_plan(lib):
+    # 32 heads, 1,048,576 tokens: 5 segments of 3276-3277 chunks
+    n, bounds = _plan(lib, 32, 1 << 20)
+    assert n == 5
+    assert np.diff(bounds).tolist() == [3277 * 64] * 4 + [3276 * 64]
+
+
+def test_plan_fits_given_scratch(lib):
+    for H in (1, 2, 3, 4, 8, 16, 32):
+        for ws in (0, 3 * H * SLOT, 16 << 20, _native.SIZE_MAX):
+            n, bounds = _plan(lib, H, 1 << 20, ws=ws)
+            _check(H, 1 << 20, n, bounds, SMS, ws)
+        assert _plan(lib, H, 1 << 20, ws=3 * H * SLOT - 1)[0] == 0   # below one split
+
+
+def test_short_and_fp32_cases_do_not_split(lib):
+    assert _plan(lib, 32, 64 * 47)[0] == 0      # fewer than 3 x 16 chunks
+    assert _plan(lib, 32, 63)[0] == 0           # shorter than one chunk: CUDA-core kernel
+    assert _plan(lib, 100, 1 << 20)[0] == 0     # 2 x 100 heads exceed one wave
+    assert lib.kda_chunk_fwd_split_plan(0, 100, SMS, 0, None) == _native.KDA_ERR_SHAPE

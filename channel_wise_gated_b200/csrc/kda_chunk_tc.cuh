@@ -276,6 +276,35 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   return make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
                     pack_bf16(v[6], v[7]));
 }
+// A 32 x 32 block of an fp32 TMEM region whose lanes index the columns of a bf16 tile
+// and whose TMEM columns index its rows: TMEM lanes lane0 .. lane0+31 (the calling
+// warp's quarter) x TMEM columns from taddr, written transposed into rows row0 ..
+// row0+31 of a K-major tile with 128-byte swizzle (64 columns per block of
+// kb_stride bytes), rounded to nearest even. Two fragment loads and four
+// transposing matrix stores of 16-byte rows per warp.
+__device__ __forceinline__ void tmem_block_to_tile_t(uint32_t taddr, int lane0, int row0,
+                                                     uint8_t* tile, uint32_t kb_stride, int lane) {
+  uint32_t v[2][16];
+  tmem_ld16x256b_x4(taddr, v[0]);
+  tmem_ld16x256b_x4(taddr + (16u << 16), v[1]);
+  tmem_ld_wait();
+  const int mi = lane >> 3;   // the matrix whose row address this thread gives
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int rp = 0; rp < 2; ++rp) {
+      const uint32_t* w = v[hf] + 8 * rp;
+      const int col = lane0 + 16 * hf + 8 * (mi & 1);       // first tile column of matrix mi
+      const int row = row0 + 8 * (2 * rp + (mi >> 1)) + (lane & 7);
+      const uint32_t addr =
+          smem_u32(tile + (col >> 6) * kb_stride) + swz128((uint32_t)row * 128u + (uint32_t)(col & 63) * 2u);
+      stmatrix_x4_trans(addr, pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                        pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                        pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                        pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7])));
+    }
+}
+
 __device__ __forceinline__ uint64_t kdesc128(uint32_t addr) {
   return make_sdesc(addr, 16, 1024, SWZ_128B);
 }
@@ -1135,15 +1164,8 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   auto w_readout = [&](int cc) -> bool {
     if (!wait_b(x, B_WDONE, cc & 1)) return false;
     tc_fence_after();
-    uint8_t* wt = x.sm + OFF_KQ + (cc % 3) * KQ_BYTES + ((cc & 1) ? 8192 : 0) + (j >> 6) * 16384;
-    const uint32_t cb = (uint32_t)(j & 63) * 2u;
-    float v[32];
-    tmem_ld32(x.tmem + TM_W + lb + 32 * hh, v);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      *reinterpret_cast<__nv_bfloat16*>(wt + swz128((32 * hh + i) * 128 + cb)) =
-          __float2bfloat16_rn(v[i]);
+    tmem_block_to_tile_t(x.tmem + TM_W + lb + 32 * hh, 32 * qd, 32 * hh,
+                         x.sm + OFF_KQ + (cc % 3) * KQ_BYTES + ((cc & 1) ? 8192 : 0), 16384u, lane);
     fence_proxy_async_smem();
     tc_fence_before();
     return true;
@@ -1203,14 +1225,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         if (L == CHUNK) {
           // full chunk: into the output tile (its previous store has read it), then one
           // TMA store of [64 rows][128 columns]
-          float v[32];
-          tmem_ld32(x.tmem + ro + lb + 32 * hh, v);
-          tmem_ld_wait();
-          uint8_t* ot = dt + (j >> 6) * 8192;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            *reinterpret_cast<__nv_bfloat16*>(ot + swz128((32 * hh + i) * 128 + (j & 63) * 2)) =
-                __float2bfloat16_rn(v[i]);
+          tmem_block_to_tile_t(x.tmem + ro + lb + 32 * hh, 32 * qd, 32 * hh, dt, 8192u, lane);
           fence_proxy_async_smem();
         } else {
           // ragged last chunk of a sequence: direct stores of the valid rows only

@@ -278,6 +278,31 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+// 16 lanes x 32 columns (four 8-column repetitions) in the mma fragment layout: for
+// repetition k, thread t holds registers 4k..4k+3 = (lane t/4, column 8k + 2(t%4)),
+// (lane t/4, column 8k + 2(t%4) + 1), and the same two columns of lane 8 + t/4
+// (lanes relative to the address's lane field). Checked on B200 with a probe that
+// loads known values.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+// Four 8x8 b16 matrices stored transposed: register m of thread t holds row t/4,
+// columns 2(t%4) and 2(t%4)+1 (low half first) of matrix m; the element in row a,
+// column b lands in row b, position a of the stored matrix, whose 8 rows (16 bytes
+// each) start at the addresses given by threads 8m .. 8m+7.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t q0, uint32_t q1,
+                                                  uint32_t q2, uint32_t q3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(q0), "r"(q1), "r"(q2), "r"(q3)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }

@@ -46,6 +46,10 @@ def load_library(path: str):
     f.restype = ctypes.c_int
     f.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int64] * 6 + [
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    g = lib.gdn_oracle_forward
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int64] * 6 + [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.kda_oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -140,3 +144,36 @@ def oracle_decode_steps(q, k, v, log_alpha, beta, state, n_threads: int = 0, col
                            h0=state, cu_seqlens=cu, n_threads=n_threads, col_block=col_block)
     o = np.swapaxes(o.reshape(N, steps, H, dv), 0, 1)
     return np.ascontiguousarray(o), hT
+
+
+def oracle_gdn_forward(q, k, v, log_a, beta, h0=None, cu_seqlens=None, n_threads: int = 0,
+                       col_block: int = 0, lib=None):
+    """Gated DeltaNet (one scalar gate per token and head) for every (sequence, head).
+
+    q, k: [T, H, dk]; v: [T, H, dv]; log_a, beta: [T, H]; h0: [N, H, dk, dv] or None;
+    cu_seqlens: [N+1] or None. Returns (o [T, H, dv] fp64, hT [N, H, dk, dv] fp64).
+    """
+    q, k, v, la, b = (_f32(x) for x in (q, k, v, log_a, beta))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    assert k.shape == (T, H, dk) and la.shape == (T, H)
+    assert v.shape == (T, H, dv) and b.shape == (T, H)
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+    N = cu.shape[0] - 1
+    h0_arr = None if h0 is None else _f64(h0)
+    if h0_arr is not None:
+        assert h0_arr.shape == (N, H, dk, dv)
+    o = np.zeros((T, H, dv), dtype=np.float64)
+    hT = np.zeros((N, H, dk, dv), dtype=np.float64)
+    lib = _load() if lib is None else lib
+    rc = lib.gdn_oracle_forward(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, la.ctypes.data, b.ctypes.data,
+        None if h0_arr is None else h0_arr.ctypes.data, cu.ctypes.data,
+        N, H, dk, dv, T, int(col_block), o.ctypes.data, hT.ctypes.data, int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"gdn_oracle_forward failed with status {rc}")
+    return o, hT

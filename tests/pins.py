@@ -192,3 +192,94 @@ def pin_contraction(fwd, seed=9, T=40):
 ALL_PINS = [pin_decay_table, pin_deltanet, pin_gated_deltanet, pin_identity_step,
             pin_pure_decay, pin_reaches_target, pin_gla_limit, pin_unrolled,
             pin_square_state_unrolled, pin_contraction]
+
+
+# ---------------------------------------------------------------------------
+# Pins for the Gated DeltaNet oracle (one scalar gate a_t per token and head;
+# "Rationalist Deep-Dive" section 2.3, summary section 2.2). Each takes ``gfwd``
+# with the signature of ``oracle.oracle_gdn_forward``.
+# ---------------------------------------------------------------------------
+
+def _gdn_one_head(gfwd, q, k, v, beta, log_a, S0=None):
+    o, hT = gfwd(q[:, None, :], k[:, None, :], v[:, None, :], log_a[:, None], beta[:, None],
+                 h0=None if S0 is None else S0[None, None])
+    return o[:, 0, :], hT[0, 0]
+
+
+def _gdn_draw(rng, T, dk, dv):
+    q, k, v, beta, _, S0 = _draw(rng, T, dk, dv)
+    log_a = np.asarray(-rng.random(T) * 0.7, dtype=np.float32).astype(np.float64)
+    return q, k, v, beta, log_a, S0
+
+
+def pin_gdn_textbook(gfwd, seed=21):
+    """Against the textbook Gated DeltaNet loop, S <- a (I - beta k k^T) S + beta k v^T."""
+    rng = np.random.default_rng(seed)
+    q, k, v, beta, log_a, S0 = _gdn_draw(rng, 12, 4, 3)
+    o, S = _gdn_one_head(gfwd, q, k, v, beta, log_a, S0)
+    o_ref, S_ref = textbook.gated_deltanet_scalar(q, k, v, beta, np.exp(log_a), S0)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_gdn_deltanet(gfwd, seed=22):
+    """a = 1 reduces Gated DeltaNet to DeltaNet (one gradient step per token)."""
+    rng = np.random.default_rng(seed)
+    q, k, v, beta, _, S0 = _gdn_draw(rng, 10, 4, 3)
+    o, S = _gdn_one_head(gfwd, q, k, v, beta, np.zeros(10), S0)
+    o_ref, S_ref = textbook.deltanet_gradient_step(q, k, v, beta, S0)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_gdn_pure_gate(gfwd, seed=23):
+    """beta = 0: S_t = a_t S_{t-1} exactly, o_t = S_t^T q_t."""
+    rng = np.random.default_rng(seed)
+    q, k, v, _, log_a, S0 = _gdn_draw(rng, 7, 4, 3)
+    o, S = _gdn_one_head(gfwd, q, k, v, np.zeros(7), log_a, S0)
+    S_ref = S0.copy()
+    for t in range(7):
+        S_ref = np.exp(log_a[t]) * S_ref
+        np.testing.assert_allclose(o[t], S_ref.T @ q[t], rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-13, atol=1e-15)
+
+
+def pin_gdn_reaches_target(gfwd, seed=24):
+    """beta = 1 and a unit key: after each token S_t^T k_t = v_t (the gated erase removes
+    the old value along k completely, then the write puts v_t there)."""
+    rng = np.random.default_rng(seed)
+    q, k, v, _, log_a, S0 = _gdn_draw(rng, 6, 4, 3)
+    for t in range(1, 7):
+        _, S = _gdn_one_head(gfwd, q[:t], k[:t], v[:t], np.ones(t), log_a[:t], S0)
+        np.testing.assert_allclose(S.T @ k[t - 1], v[t - 1], rtol=0,
+                                   atol=1e-6 * (1 + np.abs(v[t - 1]).max()))
+
+
+def pin_gdn_heads_and_sequences(gfwd, seed=25):
+    """Several heads and a packed batch: each (sequence, head) equals its own textbook
+    loop (catches a gate read from the wrong token or head)."""
+    rng = np.random.default_rng(seed)
+    H, dk, dv, lens = 3, 4, 3, [5, 0, 7]
+    T = sum(lens)
+    f = lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)
+    q = f(rng.standard_normal((T, H, dk)))
+    k = rng.standard_normal((T, H, dk))
+    k = f(k / np.linalg.norm(k, axis=2, keepdims=True))
+    v = f(rng.standard_normal((T, H, dv)))
+    beta = f(1.0 / (1.0 + np.exp(-rng.standard_normal((T, H)))))
+    log_a = f(-rng.random((T, H)) * 0.9)
+    h0 = 0.3 * rng.standard_normal((len(lens), H, dk, dv))
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    o, hT = gfwd(q, k, v, log_a, beta, h0=h0, cu_seqlens=cu)
+    for n in range(len(lens)):
+        a, b = cu[n], cu[n + 1]
+        for h in range(H):
+            o_ref, S_ref = textbook.gated_deltanet_scalar(q[a:b, h], k[a:b, h], v[a:b, h],
+                                                          beta[a:b, h], np.exp(log_a[a:b, h]),
+                                                          h0[n, h])
+            np.testing.assert_allclose(o[a:b, h], o_ref, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(hT[n, h], S_ref, rtol=1e-12, atol=1e-12)
+
+
+ALL_GDN_PINS = [pin_gdn_textbook, pin_gdn_deltanet, pin_gdn_pure_gate, pin_gdn_reaches_target,
+                pin_gdn_heads_and_sequences]

@@ -132,12 +132,36 @@ MUTANTS = {
 }
 
 
+# Mistakes planted into the Gated DeltaNet chain (the scalar gate commutes with the
+# erase, so the order of those two is not a mistake; the others are).
+_GATE = ("    for (int64_t c = 0; c < dk; ++c)\n"
+         "      for (int64_t j = 0; j < nc; ++j) S[c * nc + j] *= at;\n")
+GDN_MUTANTS = {
+    "gdn_no_exp_on_gate": [("const double at = exp((double)log_a[t * n_heads + h]);",
+                            "const double at = 1.0 + (double)log_a[t * n_heads + h];")],
+    "gdn_gate_dropped": [(_GATE, "")],
+    "gdn_gate_after_write": [(_GATE, ""), ("    /* 4. read: o_t = S^T q_t */\n",
+                                           _GATE + "    /* 4. read: o_t = S^T q_t */\n")],
+    "gdn_gate_of_next_token": [("exp((double)log_a[t * n_heads + h])",
+                                "exp((double)log_a[(t + 1 < eos ? t + 1 : t) * n_heads + h])")],
+    "gdn_erase_sign": [("S[c * nc + j] -= bk * u[j];", "S[c * nc + j] += bk * u[j];")],
+}
+
+_GDN_MARK = "static int run_gdn_chain("
+
+
 @functools.lru_cache(maxsize=None)
 def _mutant_lib(name):
     src = open(os.path.join(os.path.dirname(oracle.__file__), "kda_oracle.c")).read()
-    for old, new in MUTANTS[name]:
-        assert src.count(old) == 1, f"mutation anchor not unique/present for {name}: {old!r}"
-        src = src.replace(old, new)
+    # KDA mistakes go into the KDA chain only, Gated DeltaNet ones into its chain only
+    cut = src.index(_GDN_MARK)
+    head, tail = src[:cut], src[cut:]
+    gdn = name in GDN_MUTANTS
+    part = tail if gdn else head
+    for old, new in (GDN_MUTANTS if gdn else MUTANTS)[name]:
+        assert part.count(old) == 1, f"mutation anchor not unique/present for {name}: {old!r}"
+        part = part.replace(old, new)
+    src = head + part if gdn else part + tail
     d = tempfile.mkdtemp(prefix=f"kda_mut_{name}_")
     c = os.path.join(d, "m.c")
     so = os.path.join(d, "m.so")
@@ -163,3 +187,42 @@ def test_each_planted_mistake_fails_a_pin(name):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, f"mutant {name} passed every pin"
+
+
+@pytest.mark.parametrize("pin", pins.ALL_GDN_PINS, ids=lambda p: p.__name__)
+def test_gdn_oracle_pin(pin):
+    pin(oracle.oracle_gdn_forward)
+
+
+def test_gdn_equals_kda_with_a_shared_gate():
+    """A scalar gate is KDA's channel-wise gate with every channel equal (the scalar
+    commutes with the erase): the two oracles agree on a 128-dimensional head."""
+    rng = np.random.default_rng(26)
+    T, H, d = 40, 2, 128
+    f = lambda a: np.asarray(a, dtype=np.float32)
+    q = rng.standard_normal((T, H, d))
+    k = rng.standard_normal((T, H, d))
+    q, k = f(q / np.linalg.norm(q, axis=2, keepdims=True)), f(k / np.linalg.norm(k, axis=2, keepdims=True))
+    v = f(rng.standard_normal((T, H, d)))
+    beta = f(1.0 / (1.0 + np.exp(-rng.standard_normal((T, H)))))
+    log_a = f(-rng.random((T, H)) * 0.3)
+    h0 = 0.02 * rng.standard_normal((1, H, d, d))
+    o_g, h_g = oracle.oracle_gdn_forward(q, k, v, log_a, beta, h0=h0)
+    o_k, h_k = oracle.oracle_forward(q, k, v, np.repeat(log_a[:, :, None], d, axis=2), beta, h0=h0)
+    np.testing.assert_allclose(o_g, o_k, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(h_g, h_k, rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("name", sorted(GDN_MUTANTS))
+def test_each_planted_gdn_mistake_fails_a_pin(name):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    lib = _mutant_lib(name)
+    gfwd = functools.partial(oracle.oracle_gdn_forward, lib=lib)
+    failed = []
+    for pin in pins.ALL_GDN_PINS:
+        try:
+            pin(gfwd)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name} passed every Gated DeltaNet pin"

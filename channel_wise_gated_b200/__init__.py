@@ -50,6 +50,63 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _prefill_args(q, k, v, gate, gate_shape_tail, beta, h0, cu_seqlens, o, hT,
+                  output_final_state):
+    """Check a prefill call's tensors and allocate missing outputs; returns the
+    pointer tuple of the C prefill entry points and (o, hT, N, T, H)."""
+    if q.dim() != 3 or q.shape[2] != D:
+        raise ValueError("q must be [T, H, 128]")
+    T, H, _ = q.shape
+    dev = q.device
+    if q.dtype not in _DT:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, (T, H, D), dev)
+    _need(gate, "log gate", torch.float32, (T, H) + gate_shape_tail, dev)
+    _need(beta, "beta", torch.float32, (T, H), dev)
+    if cu_seqlens is None:
+        N = 1
+    else:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+            raise ValueError("cu_seqlens must be [N+1]")
+        N = cu_seqlens.numel() - 1
+    if h0 is not None:
+        _need(h0, "h0", torch.float32, (N, H, D, D), dev)
+    if o is None:
+        o = torch.empty_like(q)
+    else:
+        _need(o, "o", q.dtype, (T, H, D), dev)
+    if output_final_state and hT is None:
+        hT = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
+    elif hT is not None:
+        _need(hT, "hT", torch.float32, (N, H, D, D), dev)
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
+            N, T, H, _DT[q.dtype], _ptr(o), _ptr(hT))
+    return args, (o, hT, N, T, H)
+
+
+def gdn_chunk_fwd(q, k, v, log_a, beta, h0=None, cu_seqlens=None, o=None, hT=None,
+                  output_final_state: bool = True, split: bool = True):
+    """Chunkwise Gated DeltaNet prefill: KDA with one scalar gate per token and head.
+
+    q, k, v: [T, H, 128] bf16 or fp32; log_a: [T, H] fp32 (log of the gate);
+    beta: [T, H] fp32; h0, cu_seqlens, o, hT: as chunk_fwd. With ``split`` a single
+    long bf16 sequence is split in time over a workspace allocated here.
+    """
+    lib = _native.load()
+    args, (o, hT, N, T, H) = _prefill_args(q, k, v, log_a, (), beta, h0, cu_seqlens, o, hT,
+                                           output_final_state)
+    ws_bytes = 0
+    if split:
+        ws_bytes = lib.kda_chunk_fwd_workspace_size(N, T, H, _DT[q.dtype],
+                                                    int(cu_seqlens is not None))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device) if ws_bytes else None
+    st = lib.kda_gdn_chunk_fwd_ws(*args, _ptr(ws), ws_bytes, _stream_ptr(q.device))
+    _native.check(st, "kda_gdn_chunk_fwd_ws")
+    return o, hT
+
+
 def chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, o=None, hT=None,
               output_final_state: bool = True, kernel: str = "auto"):
     """Chunkwise KDA prefill.

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "../../include/kda.h"
@@ -46,17 +47,17 @@ int validate_chunk_args(const void* q, const void* k, const void* v, const float
   return KDA_OK;
 }
 
-template <typename TQ>
+template <typename TQ, bool SG>
 int launch_chunk_simt(const void* q, const void* k, const void* v, const float* log_alpha,
                       const float* beta, const float* h0, const int32_t* cu_seqlens,
                       int32_t n_seqs, int64_t t_total, int32_t n_heads, void* o, float* hT,
                       cudaStream_t stream) {
   const size_t smem = sizeof(kda::SimtSmem);
-  if (cudaFuncSetAttribute(kda::kda_chunk_simt_kernel<TQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(kda::kda_chunk_simt_kernel<TQ, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return KDA_ERR_CUDA;
   dim3 grid((unsigned)(n_seqs * n_heads), kda::D / kda::SIMT_DV);
-  kda::kda_chunk_simt_kernel<TQ><<<grid, kda::SIMT_THREADS, smem, stream>>>(
+  kda::kda_chunk_simt_kernel<TQ, SG><<<grid, kda::SIMT_THREADS, smem, stream>>>(
       static_cast<const TQ*>(q), static_cast<const TQ*>(k), static_cast<const TQ*>(v), log_alpha,
       beta, h0, cu_seqlens, n_seqs, t_total, n_heads, static_cast<TQ*>(o), hT);
   return launch_status();
@@ -65,12 +66,16 @@ int launch_chunk_simt(const void* q, const void* k, const void* v, const float* 
 int chunk_simt_dispatch(const void* q, const void* k, const void* v, const float* log_alpha,
                         const float* beta, const float* h0, const int32_t* cu_seqlens,
                         int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
-                        void* o, float* hT, cudaStream_t stream) {
+                        void* o, float* hT, bool sg, cudaStream_t stream) {
   if (qkv_dtype == KDA_F32)
-    return launch_chunk_simt<float>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
-                                    n_heads, o, hT, stream);
-  return launch_chunk_simt<__nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs,
-                                          t_total, n_heads, o, hT, stream);
+    return sg ? launch_chunk_simt<float, true>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs,
+                                               t_total, n_heads, o, hT, stream)
+              : launch_chunk_simt<float, false>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs,
+                                                t_total, n_heads, o, hT, stream);
+  return sg ? launch_chunk_simt<__nv_bfloat16, true>(q, k, v, log_alpha, beta, h0, cu_seqlens,
+                                                     n_seqs, t_total, n_heads, o, hT, stream)
+            : launch_chunk_simt<__nv_bfloat16, false>(q, k, v, log_alpha, beta, h0, cu_seqlens,
+                                                      n_seqs, t_total, n_heads, o, hT, stream);
 }
 
 // ---- tensor-core chunk kernel: TMA descriptors and launch ----
@@ -175,6 +180,7 @@ size_t order_workspace_bytes(int32_t n_seqs, int32_t n_heads) {
   return ((size_t)n_seqs * sizeof(int32_t) + 255) & ~(size_t)255;
 }
 
+template <bool SG>
 int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
                     const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                     int64_t t_total, int32_t n_heads, void* o, float* hT, int n_seg,
@@ -183,20 +189,21 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   const uint64_t cols = (uint64_t)n_heads * kda::D;
   const uint64_t rows = (uint64_t)t_total;
   CUtensorMap mk, mq, mv, mla, mo;
+  memset(&mla, 0, sizeof(mla));   // (a scalar gate has no tile map: prep A prefetches it)
   if (!encode_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, log_alpha, cols, rows, 4, 128, 64,
-                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      (!SG && !encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, log_alpha, cols, rows, 4, 128, 64,
+                         CU_TENSOR_MAP_SWIZZLE_NONE)) ||
       !encode_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return KDA_ERR_CUDA;
-  if (cudaFuncSetAttribute(kda_chunk_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(kda_chunk_tc_kernel<false, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess ||
-      cudaFuncSetAttribute(kda_chunk_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(kda_chunk_tc_kernel<true, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess)
     return KDA_ERR_CUDA;
   Args a;
@@ -224,7 +231,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   }
   if (n_seg < 3 || seg_states == nullptr) {
     const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
-    kda_chunk_tc_kernel<false><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
+    kda_chunk_tc_kernel<false, SG><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
     return launch_status();
   }
   // time split: segment states (with segment 0's output), the scan over segments,
@@ -235,7 +242,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.seg_rem = (int)(n_chunks % n_seg);
   a.seg_states = seg_states;
   a.plan = PLAN_STATES;
-  kda_chunk_tc_kernel<true><<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
+  kda_chunk_tc_kernel<true, SG><<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
   if (cudaFuncSetAttribute(kda::seg::kda_segment_scan_kernel,
@@ -246,7 +253,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
                                        stream>>>(seg_states, n_heads, n_seg);
   if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
   a.plan = PLAN_OUTPUTS;
-  kda_chunk_tc_kernel<false><<<(unsigned)(n_heads * (n_seg - 1)), THREADS, SMEM_BYTES, stream>>>(
+  kda_chunk_tc_kernel<false, SG><<<(unsigned)(n_heads * (n_seg - 1)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   return launch_status();
 }
@@ -335,6 +342,35 @@ int static_scratch_address(void** out) {
   return KDA_OK;
 }
 
+// The prefill for KDA (sg = false: log_alpha [T, H, 128]) or Gated DeltaNet (sg =
+// true: one log-gate per token and head, [T, H]): validation, then the tensor-core
+// kernel (time split when the workspace allows it) or the CUDA-core kernel.
+int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* log_alpha,
+                   const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                   int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
+                   void* workspace, size_t workspace_bytes, bool sg, cudaStream_t stream) {
+  int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                               qkv_dtype, o, hT);
+  if (st != KDA_OK) return st;
+  if (workspace && !aligned16(workspace)) return KDA_ERR_ALIGN;
+  if (use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype)) {
+    const int n_seg = workspace == nullptr ? 0 : plan_segments(cu_seqlens, n_seqs, t_total, n_heads,
+                                                               qkv_dtype, workspace_bytes);
+    int32_t* order = nullptr;
+    const size_t ob = order_workspace_bytes(n_seqs, n_heads);
+    if (n_seg == 0 && cu_seqlens != nullptr && workspace != nullptr && ob > 0 && workspace_bytes >= ob)
+      order = static_cast<int32_t*>(workspace);
+    return sg ? launch_chunk_tc<true>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
+                                      n_heads, o, hT, n_seg, static_cast<float*>(workspace), order,
+                                      stream)
+              : launch_chunk_tc<false>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
+                                       n_heads, o, hT, n_seg, static_cast<float*>(workspace), order,
+                                       stream);
+  }
+  return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                             qkv_dtype, o, hT, sg, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -347,7 +383,7 @@ int kda_chunk_fwd_simt(const void* q, const void* k, const void* v, const float*
                                qkv_dtype, o, hT);
   if (st != KDA_OK) return st;
   return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
-                             qkv_dtype, o, hT, stream);
+                             qkv_dtype, o, hT, false, stream);
 }
 
 int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
@@ -391,22 +427,25 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
                      const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                      int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
                      void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
-                               qkv_dtype, o, hT);
-  if (st != KDA_OK) return st;
-  if (workspace && !aligned16(workspace)) return KDA_ERR_ALIGN;
-  if (use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype)) {
-    const int n_seg = workspace == nullptr ? 0 : plan_segments(cu_seqlens, n_seqs, t_total, n_heads,
-                                                               qkv_dtype, workspace_bytes);
-    int32_t* order = nullptr;
-    const size_t ob = order_workspace_bytes(n_seqs, n_heads);
-    if (n_seg == 0 && cu_seqlens != nullptr && workspace != nullptr && ob > 0 && workspace_bytes >= ob)
-      order = static_cast<int32_t*>(workspace);
-    return launch_chunk_tc(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads, o,
-                           hT, n_seg, static_cast<float*>(workspace), order, stream);
-  }
-  return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
-                             qkv_dtype, o, hT, stream);
+  return chunk_fwd_impl(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
+                        qkv_dtype, o, hT, workspace, workspace_bytes, false, stream);
+}
+
+int kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* log_a,
+                      const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                      int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
+                      cudaStream_t stream) {
+  return chunk_fwd_impl(q, k, v, log_a, beta, h0, cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype,
+                        o, hT, nullptr, 0, true, stream);
+}
+
+int kda_gdn_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* log_a,
+                         const float* beta, const float* h0, const int32_t* cu_seqlens,
+                         int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                         void* o, float* hT, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream) {
+  return chunk_fwd_impl(q, k, v, log_a, beta, h0, cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype,
+                        o, hT, workspace, workspace_bytes, true, stream);
 }
 
 int kda_chunk_fwd_static(const void* q, const void* k, const void* v, const float* log_alpha,

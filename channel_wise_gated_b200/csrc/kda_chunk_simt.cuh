@@ -47,7 +47,10 @@ struct SimtSmem {
   float gC[D];                 // G of the chunk's last row
 };
 
-template <typename TQ>
+// SG = true: Gated DeltaNet, one scalar gate per token and head (log_alpha [T, H]),
+// read here as the same log-decay on every channel (the scalar commutes with the
+// erase, so the chunk algebra is unchanged).
+template <typename TQ, bool SG>
 __global__ void __launch_bounds__(SIMT_THREADS, 1)
 kda_chunk_simt_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const TQ* __restrict__ v,
                   const float* __restrict__ log_alpha, const float* __restrict__ beta,
@@ -84,7 +87,7 @@ kda_chunk_simt_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const 
         const size_t g = (size_t)(t0 + r) * row_stride + (size_t)h * D + c;
         kv = to_f32(k[g]);
         qv = to_f32(q[g]);
-        lv = log_alpha[g];
+        lv = SG ? log_alpha[(size_t)(t0 + r) * n_heads + h] : log_alpha[g];
       }
       sm.K[r * SIMT_LDK + c] = kv;
       sm.Q[r * SIMT_LDK + c] = qv;

@@ -465,7 +465,7 @@ __device__ __forceinline__ void issue_gram(const Ctx& x, int g) {
 // still in shared memory. Pairwise factors are evaluated one by one, one channel
 // half at a time with G staged in prep B's workspace; A goes to that workspace, P
 // to its tile, and Rk / Rq are built about the point before the chunk.
-__device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, int c, int L,
+__device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, bool sg, int c, int L,
                                           uint8_t* kq, uint32_t koff, uint32_t qoff, uint8_t* ck,
                                           const float* betas) {
   const int tid = threadIdx.x;
@@ -487,7 +487,14 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, i
     for (int j = 0; j < 8; ++j) {
       const int64_t t = t0 + 8 * w + j;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t < x.eos) v = ldg_nc_v4(log_alpha + (size_t)t * x.rs + x.h * D + c0);
+      if (t < x.eos) {
+        if (sg) {   // one gate per token and head
+          const float a = ldg_nc_f32(log_alpha + (size_t)t * (x.rs / D) + x.h);
+          v = make_float4(a, a, a, a);
+        } else {
+          v = ldg_nc_v4(log_alpha + (size_t)t * x.rs + x.h * D + c0);
+        }
+      }
       const float lv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -598,7 +605,7 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, i
   return true;
 }
 
-template <bool RT>
+template <bool RT, bool SG>
 __device__ void prep_a_role(const Ctx& x, const Args& p) {
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
@@ -629,12 +636,25 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
     // log-decay rows 8w..8w+7 of this chunk, channels c0..c0+3 (L2-prefetched three
     // chunks ahead by the thread that loads k/q); zero past the end of the sequence
     float g2[8][4];
+    if (SG) {
+      // one gate per row (the same address for the whole warp); the rows of the chunk
+      // two ahead go to L2 now
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int64_t t = t0 + 8 * w + j;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t < x.eos) v = ldg_nc_v4(p.log_alpha + (size_t)t * x.rs + x.h * D + c0);
-      g2[j][0] = v.x; g2[j][1] = v.y; g2[j][2] = v.z; g2[j][3] = v.w;
+      for (int j = 0; j < 8; ++j) {
+        const int64_t t = t0 + 8 * w + j;
+        const float a = t < x.eos ? ldg_nc_f32(p.log_alpha + (size_t)t * p.n_heads + x.h) : 0.f;
+        g2[j][0] = a; g2[j][1] = a; g2[j][2] = a; g2[j][3] = a;
+      }
+      const int64_t tp = t0 + 2 * CHUNK + tid;
+      if (tid < CHUNK && tp < x.eos) prefetch_l2(p.log_alpha + (size_t)tp * p.n_heads + x.h);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t t = t0 + 8 * w + j;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < x.eos) v = ldg_nc_v4(p.log_alpha + (size_t)t * x.rs + x.h * D + c0);
+        g2[j][0] = v.x; g2[j][1] = v.y; g2[j][2] = v.z; g2[j][3] = v.w;
+      }
     }
     // (the reader of this beta slot, prep B three chunks back, finished before this
     // role got the Ck slot of chunk c-1)
@@ -692,10 +712,20 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
         const uint2 kr = valid ? *kp : make_uint2(0u, 0u);
         const uint2 qv = (valid && !lean_of<RT>(x)) ? *qp : make_uint2(0u, 0u);
         float e[4], f[4];
+        if (SG) {   // one factor per row
+          e[0] = ex2f(g2[j][0] - gc[0]);
+          f[0] = rcpf(e[0]);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          e[k] = ex2f(g2[j][k] - gc[k]);
-          f[k] = rcpf(e[k]);
+          for (int k = 1; k < 4; ++k) {
+            e[k] = e[0];
+            f[k] = f[0];
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            e[k] = ex2f(g2[j][k] - gc[k]);
+            f[k] = rcpf(e[k]);
+          }
         }
         const uint32_t e01 = pack_bf16(e[0], e[1]), e23 = pack_bf16(e[2], e[3]);
         *kp = make_uint2(mul_bf16x2(kr.x, e01), mul_bf16x2(kr.y, e23));
@@ -707,7 +737,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
                          mul_bf16x2(kr.y, pack_bf16(f[2], f[3])));
       }
     } else {
-      ok = prep_a_exact(x, p.log_alpha, c, L, kq, koff, qoff, ck, betas);
+      ok = prep_a_exact(x, p.log_alpha, SG, c, L, kq, koff, qoff, ck, betas);
       if (!ok) break;
     }
     // per-channel scalars and the path flag of this chunk
@@ -785,7 +815,7 @@ __device__ __forceinline__ void blk_store_tb(uint8_t* tt, int a, int b, const fl
   }
 }
 
-template <bool RT>
+template <bool RT, bool SG>
 __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
                             const CUtensorMap* map_la) {
   const int tid = threadIdx.x - PB_WARP0 * 32;
@@ -811,12 +841,14 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
         if (block ? !wait_b(x, B_KQFREE + cn % 3, par) : !mbar_test_wait(fb, par)) return;
       }
       issue_kq<RT>(x, map_k, map_q, cn);
-      if (cn + 3 < x.n_chunks) tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
+      // (a scalar gate is prefetched by prep A itself)
+      if (!SG && cn + 3 < x.n_chunks)
+        tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
       ++kq_issued;
     }
   };
   if (tid == 0) {
-    for (int c = 0; c < 3 && c < x.n_chunks; ++c)
+    for (int c = 0; c < 3 && c < x.n_chunks && !SG; ++c)
       tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)c * CHUNK));
     push_kq(2, false);
   }
@@ -1295,12 +1327,15 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 
 // ============================================================================
 // kernel: one CTA per (sequence, head), or per (segment, head) of a time split.
+// SG = true: Gated DeltaNet, one scalar gate per token and head (log_alpha [T, H]):
+// prep A loads 64 gate values per chunk instead of the 64 x 128 tile and evaluates
+// each row's factor once; everything downstream is the same chunk algebra.
 // RT = false (PLAN_SEQ, PLAN_OUTPUTS): every CTA writes output, and only the full
 // form of the roles is compiled. RT = true (PLAN_STATES): each CTA's flag picks the
 // lean or the full form at run time, in one body of code, so that the SMs of a TPC,
 // which share instruction caches, fetch the same code whichever CTAs they hold.
 // ============================================================================
-template <bool RT>
+template <bool RT, bool SG>
 __global__ void __launch_bounds__(THREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_la,
@@ -1381,7 +1416,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   if (threadIdx.x == 0) {
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_q);
-    prefetch_tensormap(&map_la);
+    if (!SG) prefetch_tensormap(&map_la);
   }
   if (warp == ST_WARP0) {
     if (lane == 0) {
@@ -1397,9 +1432,9 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.tmem = *tmem_slot;
 
   if (warp < PA_WARPS) {
-    prep_a_role<RT>(x, args);
+    prep_a_role<RT, SG>(x, args);
   } else if (warp < ST_WARP0) {
-    prep_b_role<RT>(x, &map_k, &map_q, &map_la);
+    prep_b_role<RT, SG>(x, &map_k, &map_q, &map_la);
   } else {
     state_role<RT>(x, args, &map_v, &map_o);
   }

@@ -213,6 +213,39 @@ int kda_chunk_fwd_simt(const void* q, const void* k, const void* v, const float*
                        void* o, float* hT, cudaStream_t stream);
 
 /*
+ * kda_gdn_chunk_fwd - chunkwise prefill of Gated DeltaNet, the scalar-gate
+ * specialisation of the same operator (Rationalist Deep-Dive, section 2.3
+ * "Gated DeltaNet: The Scalar Forget"; Kimi Linear summary, section 2.2):
+ *
+ *     S_t = a_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t
+ *
+ * with ONE gate a_t in (0, 1] per token and head instead of KDA's 128 per-channel
+ * gates. The scalar commutes with the erase, so this is exactly KDA with the same
+ * log-decay on every channel; the kernels read 64 gate values per chunk instead of
+ * a 64 x 128 tile (4 bytes per token and head instead of 512) and evaluate each
+ * row's decay factor once. The Summary's efficiency comparison (section 5.6) puts
+ * the two gates side by side; this entry point lets a caller do the same.
+ *
+ * Arguments, layouts, chunking, precision and errors: as kda_chunk_fwd, except
+ *   log_a   [t_total, n_heads] fp32, log a_t (finite, <= 0)
+ */
+int kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* log_a,
+                      const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
+                      int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype, void* o, float* hT,
+                      cudaStream_t stream);
+
+/*
+ * kda_gdn_chunk_fwd_ws - kda_gdn_chunk_fwd with a caller-provided workspace for the
+ * time split of one long bf16 sequence, exactly as kda_chunk_fwd_ws (same plan,
+ * same workspace size: kda_chunk_fwd_workspace_size).
+ */
+int kda_gdn_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* log_a,
+                         const float* beta, const float* h0, const int32_t* cu_seqlens,
+                         int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                         void* o, float* hT, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/*
  * kda_decode_step - one recurrent KDA update per (sequence, head), in place.
  *
  * For each of the n_seqs * n_heads states (section 6.3 "Complexity Analysis":

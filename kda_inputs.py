@@ -96,12 +96,14 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
 
 def make_prefill(lens, n_heads: int, qkv_dtype=torch.bfloat16, gate_dtype=torch.float32,
                  x_mean: float = 3.0, h0: bool = False, seed: int = 0, device="cpu",
-                 slab: int = 1 << 16, d: int = D, h0_std: float = 0.02):
+                 slab: int = 1 << 16, d: int = D, h0_std: float = 0.02,
+                 scalar_gate: bool = False):
     """Draw a packed prefill batch.
 
     Returns a dict with q, k, v [T, H, d] (qkv_dtype), log_alpha [T, H, d] and
     beta [T, H] (gate_dtype), h0 [N, H, d, d] fp32 or None, cu_seqlens [N+1] int32
-    and lens (list).
+    and lens (list). With scalar_gate the log-decay is one value per token and head,
+    log_alpha [T, H] (the Gated DeltaNet gate), drawn the same way.
     """
     lens = [int(x) for x in lens]
     T = sum(lens)
@@ -110,7 +112,8 @@ def make_prefill(lens, n_heads: int, qkv_dtype=torch.bfloat16, gate_dtype=torch.
     q = torch.empty((T, n_heads, d), dtype=qkv_dtype, device=device)
     k = torch.empty_like(q)
     v = torch.empty_like(q)
-    la = torch.empty((T, n_heads, d), dtype=gate_dtype, device=device)
+    la = torch.empty((T, n_heads) if scalar_gate else (T, n_heads, d), dtype=gate_dtype,
+                     device=device)
     b = torch.empty((T, n_heads), dtype=gate_dtype, device=device)
     for t0 in range(0, T, slab):
         t1 = min(T, t0 + slab)
@@ -118,7 +121,7 @@ def make_prefill(lens, n_heads: int, qkv_dtype=torch.bfloat16, gate_dtype=torch.
         q[t0:t1] = _unit_rows(torch.randn(shp, generator=g, device=device)).to(qkv_dtype)
         k[t0:t1] = _unit_rows(torch.randn(shp, generator=g, device=device)).to(qkv_dtype)
         v[t0:t1] = torch.randn(shp, generator=g, device=device).to(qkv_dtype)
-        x = torch.randn(shp, generator=g, device=device) + x_mean
+        x = torch.randn(shp[:2] if scalar_gate else shp, generator=g, device=device) + x_mean
         la[t0:t1] = torch.nn.functional.logsigmoid(x).to(gate_dtype)
         b[t0:t1] = torch.sigmoid(torch.randn(shp[:2], generator=g, device=device)).to(gate_dtype)
     h0_t = None

@@ -9,6 +9,10 @@ and of its scalar-gate relative, Gated DeltaNet (Rationalist Deep-Dive, section 
 
     S_t = a_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
 
+and of the general DPLR recurrence it specialises (Deep-Dive, section 3.2):
+
+    S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} + k_t v_t^T
+
 Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package. The product path (the CUDA library and
 its Python binding) never imports, links or calls anything here, and this
@@ -20,6 +24,7 @@ from .kda_oracle import (  # noqa: F401
     load_library,
     oracle_forward,
     oracle_gdn_forward,
+    oracle_dplr_forward,
     oracle_decode_steps,
     oracle_threads,
 )

@@ -50,6 +50,10 @@ def load_library(path: str):
     g.restype = ctypes.c_int
     g.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int64] * 6 + [
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    dp = lib.dplr_oracle_forward
+    dp.restype = ctypes.c_int
+    dp.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 6 + [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.kda_oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -176,4 +180,34 @@ def oracle_gdn_forward(q, k, v, log_a, beta, h0=None, cu_seqlens=None, n_threads
         N, H, dk, dv, T, int(col_block), o.ctypes.data, hT.ctypes.data, int(n_threads))
     if rc != 0:
         raise RuntimeError(f"gdn_oracle_forward failed with status {rc}")
+    return o, hT
+
+
+def oracle_dplr_forward(q, k, v, a, b, log_alpha, h0=None, cu_seqlens=None, n_threads: int = 0,
+                        col_block: int = 0, lib=None):
+    """General DPLR recurrence S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} + k_t v_t^T for every
+    (sequence, head). q, k, a, b, log_alpha: [T, H, dk]; v: [T, H, dv]; h0, cu_seqlens as
+    oracle_forward. Returns (o [T, H, dv] fp64, hT [N, H, dk, dv] fp64)."""
+    q, k, v, a, b, la = (_f32(x) for x in (q, k, v, a, b, log_alpha))
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    for x in (k, a, b, la):
+        assert x.shape == (T, H, dk)
+    assert v.shape == (T, H, dv)
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+    N = cu.shape[0] - 1
+    h0_arr = None if h0 is None else _f64(h0)
+    o = np.zeros((T, H, dv), dtype=np.float64)
+    hT = np.zeros((N, H, dk, dv), dtype=np.float64)
+    lib = _load() if lib is None else lib
+    rc = lib.dplr_oracle_forward(
+        q.ctypes.data, k.ctypes.data, v.ctypes.data, a.ctypes.data, b.ctypes.data, la.ctypes.data,
+        None if h0_arr is None else h0_arr.ctypes.data, cu.ctypes.data,
+        N, H, dk, dv, T, int(col_block), o.ctypes.data, hT.ctypes.data, int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"dplr_oracle_forward failed with status {rc}")
     return o, hT

@@ -108,14 +108,15 @@ def short_conv_swish(x, w, cu_seqlens=None):
 
 def fused_layer_forward(q_pre, k_pre, v_pre, decay_pre, beta_pre, gate_pre, norm_weight,
                         h0=None, cu_seqlens=None, conv_w=None, n_threads: int = 0,
-                        col_block: int = 0):
+                        col_block: int = 0, return_pre_norm: bool = False):
     """The recurrence with the operations around it, in the order the pages give.
 
     q_pre, k_pre, v_pre: [T, H, 128] (the projections' outputs); decay_pre: [T, H, 128]
     (log alpha = logsigmoid(decay_pre)); beta_pre: [T, H] (beta = sigmoid(beta_pre));
     gate_pre: [T, H, 128]; norm_weight: [128]; conv_w: None, or a dict with "q", "k", "v"
     filters [H * 128, 4] (short convolution + Swish before the rest). Returns
-    (o_final [T, H, 128], hT [N, H, 128, 128]) in fp64.
+    (o_final [T, H, 128], hT [N, H, 128, 128]) in fp64, and with return_pre_norm also
+    the recurrence's output o before the RMSNorm.
 
     The recurrence itself is the C oracle (kda_oracle.c), which reads its inputs as
     fp32: the fp64 results of the steps before it are rounded to fp32 there (a relative
@@ -135,4 +136,6 @@ def fused_layer_forward(q_pre, k_pre, v_pre, decay_pre, beta_pre, gate_pre, norm
     beta = sigmoid(beta_pre)
     o, hT = oracle_forward(q, k, v, log_alpha, beta, h0=h0, cu_seqlens=cu_seqlens,
                            n_threads=n_threads, col_block=col_block)
+    if return_pre_norm:
+        return output_gate(o, norm_weight, gate_pre), hT, o
     return output_gate(o, norm_weight, gate_pre), hT

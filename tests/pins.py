@@ -283,3 +283,64 @@ def pin_gdn_heads_and_sequences(gfwd, seed=25):
 
 ALL_GDN_PINS = [pin_gdn_textbook, pin_gdn_deltanet, pin_gdn_pure_gate, pin_gdn_reaches_target,
                 pin_gdn_heads_and_sequences]
+
+
+# ---------------------------------------------------------------------------
+# Pins for the general DPLR oracle (Rationalist Deep-Dive, section 3.2; summary
+# section 6.2). Each takes ``dfwd`` with the signature of ``oracle.oracle_dplr_forward``.
+# ---------------------------------------------------------------------------
+
+def _dplr_one_head(dfwd, q, k, v, a, b, log_alpha, S0=None):
+    o, hT = dfwd(q[:, None], k[:, None], v[:, None], a[:, None], b[:, None],
+                 log_alpha[:, None], h0=None if S0 is None else S0[None, None])
+    return o[:, 0], hT[0, 0]
+
+
+def _dplr_draw(rng, T, dk, dv):
+    q, k, v, _, la, S0 = _draw(rng, T, dk, dv)
+    f = lambda x: np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = f(0.5 * rng.standard_normal((T, dk)) / np.sqrt(dk))
+    b = f(0.5 * rng.standard_normal((T, dk)) / np.sqrt(dk))
+    return q, k, v, a, b, la, S0
+
+
+def pin_dplr_unrolled(dfwd, seed=31):
+    """Brute force: explicit products of Diag(alpha) - a b^T (catches a transposed
+    low-rank term, a and b swapped, the read of the decayed state)."""
+    rng = np.random.default_rng(seed)
+    q, k, v, a, b, la, S0 = _dplr_draw(rng, 6, 4, 3)
+    o, S = _dplr_one_head(dfwd, q, k, v, a, b, la, S0)
+    o_ref, S_ref = textbook.dplr_unrolled(q, k, v, a, b, np.exp(la), S0)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-11, atol=1e-12)
+
+
+def pin_dplr_without_correction_is_gla(dfwd, seed=32):
+    """a = 0: no low-rank correction, the per-channel decay and an additive write (GLA)."""
+    rng = np.random.default_rng(seed)
+    q, k, v, _, b, la, S0 = _dplr_draw(rng, 9, 4, 3)
+    o, S = _dplr_one_head(dfwd, q, k, v, np.zeros_like(b), b, la, S0)
+    o_ref, S_ref = textbook.gla(q, k, v, np.exp(la), S0)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_dplr_tied_factors_are_kda(dfwd, seed=33):
+    """a = beta k, b = k * alpha and the value scaled by beta give KDA (the DPLR form of
+    the KDA update in Deep-Dive section 3.2, with beta on the write as in summary
+    section 3): the result equals the textbook KDA brute force."""
+    rng = np.random.default_rng(seed)
+    q, k, v, beta, la, S0 = _draw(rng, 7, 4, 3)
+    alpha = np.exp(la)
+    a = beta[:, None] * k
+    b = k * alpha
+    o, S = _dplr_one_head(dfwd, q, k, beta[:, None] * v, a, b, la, S0)
+    o_ref, S_ref = textbook.kda_unrolled(q, k, v, beta, alpha, S0)
+    # (a, b and beta v are formed in fp64 here and rounded to fp32 by the oracle's input
+    #  conversion: agreement to ~1e-7 relative, against O(1) for a wrong formula)
+    np.testing.assert_allclose(o, o_ref, rtol=2e-6, atol=1e-9)
+    np.testing.assert_allclose(S, S_ref, rtol=2e-6, atol=1e-9)
+
+
+ALL_DPLR_PINS = [pin_dplr_unrolled, pin_dplr_without_correction_is_gla,
+                 pin_dplr_tied_factors_are_kda]

@@ -102,3 +102,31 @@ def kda_unrolled(q, k, v, beta, alpha, S0=None):
     for i in range(T):
         S_T = S_T + prod(i + 1, T - 1) @ (beta[i] * np.outer(k[i], v[i]))
     return o, S_T
+
+
+def dplr_unrolled(q, k, v, a, b, alpha, S0=None):
+    """Brute force for the general DPLR recurrence: explicit d_k x d_k transitions
+    A_j = Diag(alpha_j) - a_j b_j^T and o_t = q_t^T [(A_t...A_1) S0 + sum_i (A_t...A_{i+1}) k_i v_i^T]
+    (Rationalist Deep-Dive, section 3.2 "DPLR Structure")."""
+    T, dk = q.shape
+    dv = v.shape[1]
+    S0 = np.zeros((dk, dv)) if S0 is None else np.array(S0, dtype=np.float64)
+    eye = np.eye(dk)
+    A = [np.diag(alpha[j]) - np.outer(a[j], b[j]) for j in range(T)]
+
+    def prod(lo, hi):
+        P = eye.copy()
+        for j in range(lo, hi + 1):
+            P = A[j] @ P
+        return P
+
+    o = np.zeros((T, dv))
+    for t in range(T):
+        M = prod(0, t) @ S0
+        for i in range(t + 1):
+            M = M + prod(i + 1, t) @ np.outer(k[i], v[i])
+        o[t] = M.T @ q[t]
+    S_T = prod(0, T - 1) @ S0
+    for i in range(T):
+        S_T = S_T + prod(i + 1, T - 1) @ np.outer(k[i], v[i])
+    return o, S_T

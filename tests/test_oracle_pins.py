@@ -148,20 +148,38 @@ GDN_MUTANTS = {
 }
 
 _GDN_MARK = "static int run_gdn_chain("
+_DPLR_MARK = "static int run_dplr_chain("
+
+# Mistakes planted into the DPLR chain.
+DPLR_MUTANTS = {
+    "dplr_ab_swapped": [("const double bc = (double)bt[c];", "const double bc = (double)at[c];"),
+                        ("const double ac = (double)at[c];", "const double ac = (double)bt[c];")],
+    "dplr_read_after_forget": [
+        ("    /* 1. low-rank read of the old state: u = b^T S */\n",
+         "    for (int64_t c = 0; c < dk; ++c) { const double al0 = exp((double)lat[c]);\n"
+         "      for (int64_t j = 0; j < nc; ++j) S[c * nc + j] *= al0; }\n"),
+        ("    /* 2. forget: S <- Diag(alpha) S */\n    for (int64_t c = 0; c < dk; ++c) {\n"
+         "      const double al = exp((double)lat[c]);\n",
+         "    for (int64_t c = 0; c < dk; ++c) {\n      const double al = 1.0;\n")],
+    "dplr_correction_sign": [("S[c * nc + j] -= ac * u[j];", "S[c * nc + j] += ac * u[j];")],
+    "dplr_no_forget": [("      const double al = exp((double)lat[c]);", "      const double al = 1.0;")],
+}
 
 
 @functools.lru_cache(maxsize=None)
 def _mutant_lib(name):
     src = open(os.path.join(os.path.dirname(oracle.__file__), "kda_oracle.c")).read()
     # KDA mistakes go into the KDA chain only, Gated DeltaNet ones into its chain only
-    cut = src.index(_GDN_MARK)
-    head, tail = src[:cut], src[cut:]
-    gdn = name in GDN_MUTANTS
-    part = tail if gdn else head
-    for old, new in (GDN_MUTANTS if gdn else MUTANTS)[name]:
+    c1, c2 = src.index(_GDN_MARK), src.index(_DPLR_MARK)
+    parts = [src[:c1], src[c1:c2], src[c2:]]   # KDA chain, Gated DeltaNet chain, DPLR chain
+    which = 1 if name in GDN_MUTANTS else (2 if name in DPLR_MUTANTS else 0)
+    table = (MUTANTS, GDN_MUTANTS, DPLR_MUTANTS)[which]
+    part = parts[which]
+    for old, new in table[name]:
         assert part.count(old) == 1, f"mutation anchor not unique/present for {name}: {old!r}"
         part = part.replace(old, new)
-    src = head + part if gdn else part + tail
+    parts[which] = part
+    src = "".join(parts)
     d = tempfile.mkdtemp(prefix=f"kda_mut_{name}_")
     c = os.path.join(d, "m.c")
     so = os.path.join(d, "m.so")
@@ -226,3 +244,23 @@ def test_each_planted_gdn_mistake_fails_a_pin(name):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, f"mutant {name} passed every Gated DeltaNet pin"
+
+
+@pytest.mark.parametrize("pin", pins.ALL_DPLR_PINS, ids=lambda p: p.__name__)
+def test_dplr_oracle_pin(pin):
+    pin(oracle.oracle_dplr_forward)
+
+
+@pytest.mark.parametrize("name", sorted(DPLR_MUTANTS))
+def test_each_planted_dplr_mistake_fails_a_pin(name):
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    lib = _mutant_lib(name)
+    dfwd = functools.partial(oracle.oracle_dplr_forward, lib=lib)
+    failed = []
+    for pin in pins.ALL_DPLR_PINS:
+        try:
+            pin(dfwd)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name} passed every DPLR pin"

@@ -51,7 +51,7 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 def _prefill_args(q, k, v, gate, gate_shape_tail, beta, h0, cu_seqlens, o, hT,
-                  output_final_state):
+                  output_final_state, check_gate=True):
     """Check a prefill call's tensors and allocate missing outputs; returns the
     pointer tuple of the C prefill entry points and (o, hT, N, T, H)."""
     if q.dim() != 3 or q.shape[2] != D:
@@ -62,7 +62,8 @@ def _prefill_args(q, k, v, gate, gate_shape_tail, beta, h0, cu_seqlens, o, hT,
         raise TypeError(f"unsupported dtype {q.dtype}")
     for name, t in (("q", q), ("k", k), ("v", v)):
         _need(t, name, q.dtype, (T, H, D), dev)
-    _need(gate, "log gate", torch.float32, (T, H) + gate_shape_tail, dev)
+    if check_gate:
+        _need(gate, "log gate", torch.float32, (T, H) + gate_shape_tail, dev)
     _need(beta, "beta", torch.float32, (T, H), dev)
     if cu_seqlens is None:
         N = 1
@@ -84,6 +85,65 @@ def _prefill_args(q, k, v, gate, gate_shape_tail, beta, h0, cu_seqlens, o, hT,
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(h0), _ptr(cu_seqlens),
             N, T, H, _DT[q.dtype], _ptr(o), _ptr(hT))
     return args, (o, hT, N, T, H)
+
+
+def short_conv_swish(x, w, cu_seqlens=None, y=None):
+    """Causal 4-tap depthwise convolution + Swish over tokens, restarted per sequence.
+
+    x: [T, H, 128] (or [T, C]) bf16; w: [C, 4] fp32 with C = H * 128; cu_seqlens:
+    [N+1] int32 on the device or None. Returns y like x.
+    """
+    lib = _native.load()
+    dev = x.device
+    T = x.shape[0]
+    C = x.numel() // max(T, 1) if T else int(torch.tensor(x.shape[1:]).prod())
+    _need(x, "x", torch.bfloat16, None, dev)
+    _need(w, "w", torch.float32, (C, 4), dev)
+    if cu_seqlens is None:
+        N = 1
+    else:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        N = cu_seqlens.numel() - 1
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        _need(y, "y", torch.bfloat16, tuple(x.shape), dev)
+    st = lib.kda_short_conv_swish(_ptr(x), _ptr(w), _ptr(cu_seqlens), N, T, C, _ptr(y),
+                                  _stream_ptr(dev))
+    _native.check(st, "kda_short_conv_swish")
+    return y
+
+
+def chunk_fwd_fused(q_pre, k_pre, v, decay_pre, beta_pre, gate_pre, norm_w, h0=None,
+                    cu_seqlens=None, o=None, hT=None, output_final_state: bool = True,
+                    split: bool = True):
+    """KDA prefill with the layer's activations and output gate fused in.
+
+    q_pre, k_pre, v, decay_pre, gate_pre: [T, H, 128] bf16; beta_pre: [T, H] fp32;
+    norm_w: [128] fp32. q and k are L2-normalised in the kernel, log alpha =
+    logsigmoid(decay_pre), beta = sigmoid(beta_pre), and the output is the head-wise
+    RMSNorm of o times norm_w times sigmoid(gate_pre). Returns (o_out, hT).
+    """
+    lib = _native.load()
+    T, H, _ = q_pre.shape
+    dev = q_pre.device
+    _need(q_pre, "q_pre", torch.bfloat16, (T, H, D), dev)
+    _need(decay_pre, "decay_pre", torch.bfloat16, (T, H, D), dev)
+    _need(gate_pre, "gate_pre", torch.bfloat16, (T, H, D), dev)
+    _need(norm_w, "norm_w", torch.float32, (D,), dev)
+    args, (o, hT, N, T, H) = _prefill_args(q_pre, k_pre, v, None, None, beta_pre, h0,
+                                           cu_seqlens, o, hT, output_final_state,
+                                           check_gate=False)
+    ws_bytes = 0
+    if split:
+        ws_bytes = lib.kda_chunk_fwd_workspace_size(N, T, H, _native.KDA_BF16,
+                                                    int(cu_seqlens is not None))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    q_, k_, v_, _, b_, h0_, cu_, N_, T_, H_, _, o_, hT_ = args
+    st = lib.kda_chunk_fwd_fused(q_, k_, v_, _ptr(decay_pre), b_, _ptr(gate_pre), _ptr(norm_w),
+                                 h0_, cu_, N_, T_, H_, o_, hT_, _ptr(ws), ws_bytes, _stream_ptr(dev))
+    _native.check(st, "kda_chunk_fwd_fused")
+    return o, hT
 
 
 def gdn_chunk_fwd(q, k, v, log_a, beta, h0=None, cu_seqlens=None, o=None, hT=None,

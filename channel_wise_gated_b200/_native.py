@@ -40,6 +40,9 @@ SIGNATURES = {
     "kda_chunk_fwd_workspace_size": [_I32, _I64, _I32, ctypes.c_int, ctypes.c_int],
     "kda_chunk_fwd_split_plan": [_I32, _I64, _I32, ctypes.c_size_t, _P],
     "kda_chunk_fwd_static": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
+    "kda_chunk_fwd_fused": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, _P, _P, _P,
+                            ctypes.c_size_t, _P],
+    "kda_short_conv_swish": [_P, _P, _P, _I32, _I64, _I32, _P, _P],
     "kda_gdn_chunk_fwd": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
     "kda_gdn_chunk_fwd_ws": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P,
                              ctypes.c_size_t, _P],

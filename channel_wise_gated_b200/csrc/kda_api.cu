@@ -13,6 +13,7 @@
 #include "kda_chunk_simt.cuh"
 #include "kda_chunk_tc.cuh"
 #include "kda_common.cuh"
+#include "kda_conv.cuh"
 #include "kda_decode.cuh"
 #include "kda_segment.cuh"
 
@@ -180,30 +181,44 @@ size_t order_workspace_bytes(int32_t n_seqs, int32_t n_heads) {
   return ((size_t)n_seqs * sizeof(int32_t) + 255) & ~(size_t)255;
 }
 
-template <bool SG>
+// The fused variant's inputs (MODE_FUSED): pre-activations and the norm weight.
+struct FusedIO {
+  const void* decay_pre;
+  const float* beta_pre;
+  const void* gate_pre;
+  const float* norm_w;
+};
+
+template <int MODE>
 int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
                     const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                     int64_t t_total, int32_t n_heads, void* o, float* hT, int n_seg,
-                    float* seg_states, int32_t* seq_order, cudaStream_t stream) {
+                    float* seg_states, int32_t* seq_order, const FusedIO* fu, cudaStream_t stream) {
   using namespace kda::tc;
   const uint64_t cols = (uint64_t)n_heads * kda::D;
   const uint64_t rows = (uint64_t)t_total;
   CUtensorMap mk, mq, mv, mla, mo;
   memset(&mla, 0, sizeof(mla));   // (a scalar gate has no tile map: prep A prefetches it)
-  if (!encode_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, cols, rows, 2, 64, 64,
+  bool la_ok = true;
+  if (MODE == MODE_KDA)
+    la_ok = encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, log_alpha, cols, rows, 4, 128, 64,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  else if (MODE == MODE_FUSED)   // the bf16 decay pre-activation, prefetched the same way
+    la_ok = encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, fu->decay_pre, cols, rows, 2, 128, 64,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!la_ok ||
+      !encode_2d(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_2d(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-      (!SG && !encode_2d(&mla, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, log_alpha, cols, rows, 4, 128, 64,
-                         CU_TENSOR_MAP_SWIZZLE_NONE)) ||
       !encode_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o, cols, rows, 2, 64, 64,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return KDA_ERR_CUDA;
-  if (cudaFuncSetAttribute(kda_chunk_tc_kernel<false, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(kda_chunk_tc_kernel<false, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess ||
-      cudaFuncSetAttribute(kda_chunk_tc_kernel<true, SG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(kda_chunk_tc_kernel<true, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_BYTES) != cudaSuccess)
     return KDA_ERR_CUDA;
   Args a;
@@ -222,6 +237,10 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.seg_rem = 0;
   a.seg_states = nullptr;
   a.seq_order = nullptr;
+  a.decay_pre = fu ? static_cast<const __nv_bfloat16*>(fu->decay_pre) : nullptr;
+  a.beta_pre = fu ? fu->beta_pre : nullptr;
+  a.gate_pre = fu ? static_cast<const __nv_bfloat16*>(fu->gate_pre) : nullptr;
+  a.norm_w = fu ? fu->norm_w : nullptr;
   if (seq_order != nullptr && cu_seqlens != nullptr && n_seqs > 1) {
     const unsigned blocks = (unsigned)((n_seqs + kda::seg::ORDER_THREADS - 1) / kda::seg::ORDER_THREADS);
     kda::seg::kda_seq_order_kernel<<<blocks, kda::seg::ORDER_THREADS, 0, stream>>>(
@@ -231,7 +250,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   }
   if (n_seg < 3 || seg_states == nullptr) {
     const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
-    kda_chunk_tc_kernel<false, SG><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
+    kda_chunk_tc_kernel<false, MODE><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
     return launch_status();
   }
   // time split: segment states (with segment 0's output), the scan over segments,
@@ -242,7 +261,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.seg_rem = (int)(n_chunks % n_seg);
   a.seg_states = seg_states;
   a.plan = PLAN_STATES;
-  kda_chunk_tc_kernel<true, SG><<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
+  kda_chunk_tc_kernel<true, MODE><<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
   if (cudaFuncSetAttribute(kda::seg::kda_segment_scan_kernel,
@@ -253,7 +272,7 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
                                        stream>>>(seg_states, n_heads, n_seg);
   if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
   a.plan = PLAN_OUTPUTS;
-  kda_chunk_tc_kernel<false, SG><<<(unsigned)(n_heads * (n_seg - 1)), THREADS, SMEM_BYTES, stream>>>(
+  kda_chunk_tc_kernel<false, MODE><<<(unsigned)(n_heads * (n_seg - 1)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   return launch_status();
 }
@@ -360,12 +379,14 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* log
     const size_t ob = order_workspace_bytes(n_seqs, n_heads);
     if (n_seg == 0 && cu_seqlens != nullptr && workspace != nullptr && ob > 0 && workspace_bytes >= ob)
       order = static_cast<int32_t*>(workspace);
-    return sg ? launch_chunk_tc<true>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
-                                      n_heads, o, hT, n_seg, static_cast<float*>(workspace), order,
-                                      stream)
-              : launch_chunk_tc<false>(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total,
-                                       n_heads, o, hT, n_seg, static_cast<float*>(workspace), order,
-                                       stream);
+    return sg ? launch_chunk_tc<kda::tc::MODE_GDN>(q, k, v, log_alpha, beta, h0, cu_seqlens,
+                                                   n_seqs, t_total, n_heads, o, hT, n_seg,
+                                                   static_cast<float*>(workspace), order, nullptr,
+                                                   stream)
+              : launch_chunk_tc<kda::tc::MODE_KDA>(q, k, v, log_alpha, beta, h0, cu_seqlens,
+                                                   n_seqs, t_total, n_heads, o, hT, n_seg,
+                                                   static_cast<float*>(workspace), order, nullptr,
+                                                   stream);
   }
   return chunk_simt_dispatch(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                              qkv_dtype, o, hT, sg, stream);
@@ -429,6 +450,61 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
                      void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   return chunk_fwd_impl(q, k, v, log_alpha, beta, h0, cu_seqlens, n_seqs, t_total, n_heads,
                         qkv_dtype, o, hT, workspace, workspace_bytes, false, stream);
+}
+
+int kda_chunk_fwd_fused(const void* q_pre, const void* k_pre, const void* v,
+                        const void* decay_pre, const float* beta_pre, const void* gate_pre,
+                        const float* norm_w, const float* h0, const int32_t* cu_seqlens,
+                        int32_t n_seqs, int64_t t_total, int32_t n_heads, void* o, float* hT,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  // (beta_pre is checked as beta is; decay_pre and gate_pre below)
+  int st = validate_chunk_args(q_pre, k_pre, v, static_cast<const float*>(decay_pre), beta_pre, h0,
+                               cu_seqlens, n_seqs, t_total, n_heads, KDA_BF16, o, hT);
+  if (st != KDA_OK) return st;
+  if (t_total > 0 && (!gate_pre || !norm_w)) return KDA_ERR_NULL;
+  if ((gate_pre && !aligned16(gate_pre)) || (norm_w && !aligned16(norm_w))) return KDA_ERR_ALIGN;
+  if (workspace && !aligned16(workspace)) return KDA_ERR_ALIGN;
+  if (t_total == 0) {   // nothing to compute: the final state is the initial one
+    if (hT != nullptr) {
+      const size_t bytes = (size_t)n_seqs * n_heads * kda::D * kda::D * sizeof(float);
+      const cudaError_t e = h0 ? cudaMemcpyAsync(hT, h0, bytes, cudaMemcpyDeviceToDevice, stream)
+                               : cudaMemsetAsync(hT, 0, bytes, stream);
+      if (e != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+  }
+  if (!use_tc(cu_seqlens, n_seqs, t_total, n_heads, KDA_BF16)) return KDA_ERR_SHAPE;
+  const int n_seg = workspace == nullptr ? 0 : plan_segments(cu_seqlens, n_seqs, t_total, n_heads,
+                                                             KDA_BF16, workspace_bytes);
+  int32_t* order = nullptr;
+  const size_t ob = order_workspace_bytes(n_seqs, n_heads);
+  if (n_seg == 0 && cu_seqlens != nullptr && workspace != nullptr && ob > 0 && workspace_bytes >= ob)
+    order = static_cast<int32_t*>(workspace);
+  const FusedIO fu = {decay_pre, beta_pre, gate_pre, norm_w};
+  return launch_chunk_tc<kda::tc::MODE_FUSED>(q_pre, k_pre, v, nullptr, nullptr, h0, cu_seqlens,
+                                              n_seqs, t_total, n_heads, o, hT, n_seg,
+                                              static_cast<float*>(workspace), order, &fu, stream);
+}
+
+int kda_short_conv_swish(const void* x, const float* w, const int32_t* cu_seqlens, int32_t n_seqs,
+                         int64_t t_total, int32_t channels, void* y, cudaStream_t stream) {
+  if (t_total < 0 || channels <= 0 || (channels & 7) != 0 || n_seqs <= 0) return KDA_ERR_SHAPE;
+  if (cu_seqlens == nullptr && n_seqs != 1) return KDA_ERR_SEQLENS;
+  if (t_total == 0) return KDA_OK;
+  if (!x || !w || !y) return KDA_ERR_NULL;
+  const void* ptrs[] = {x, w, y, cu_seqlens};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_ALIGN;
+  if (x == y) return KDA_ERR_SHAPE;   // (no in-place: runs read the rows before them)
+  using namespace kda::conv;
+  const int64_t runs = (t_total + CONV_RUN - 1) / CONV_RUN;
+  const int64_t threads = runs * (channels / 8);
+  const int64_t blocks = (threads + CONV_THREADS - 1) / CONV_THREADS;
+  if (blocks > (int64_t)INT32_MAX) return KDA_ERR_SHAPE;
+  kda_short_conv_swish_kernel<<<(unsigned)blocks, CONV_THREADS, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), w, cu_seqlens, n_seqs, t_total, channels,
+      static_cast<__nv_bfloat16*>(y));
+  return launch_status();
 }
 
 int kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* log_a,

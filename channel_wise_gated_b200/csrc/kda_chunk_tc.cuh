@@ -76,6 +76,18 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float GUARD_LOG2 = 60.0f * 1.4426950408889634f;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 
+// What the kernel reads and writes around the recurrence:
+//   MODE_KDA    q, k (unit length), v, log_alpha [T, H, 128] fp32, beta [T, H] fp32 -> o
+//   MODE_GDN    the same with one log-gate per token and head, log_alpha [T, H]
+//   MODE_FUSED  the producing layer's activations and the output's post-processing
+//               fused in: q and k are L2-normalised in the loader, the decay arrives
+//               as a bf16 pre-activation x (log alpha = logsigmoid(x)), beta as a
+//               pre-activation (sigmoid), and the output leaves as head-wise RMSNorm
+//               times a weight times sigmoid(gate pre-activation)
+enum : int { MODE_KDA = 0, MODE_GDN = 1, MODE_FUSED = 2 };
+constexpr float L2_EPS = 1e-12f;   // guards the L2 normalisation of an all-zero row
+constexpr float RMS_EPS = 1e-6f;   // RMSNorm epsilon
+
 // ---- shared memory layout (offsets from a 1024-byte aligned base) ----
 // Stage tile: 2 kblocks (channels 0-63, 64-127) x [128 rows][128 B], 128B swizzle.
 // Rows 0-63 / 64-127 hold k (then Rk, then -W') and q (then Rq): k on top for even
@@ -99,7 +111,9 @@ constexpr uint32_t OFF_XFLAG = OFF_GROW + 2 * 128 * 4; // [3] exact-path flag pe
 constexpr uint32_t OFF_BAR = OFF_XFLAG + 16;
 constexpr int NBARS = 32;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
-constexpr uint32_t SMEM_USED = OFF_MISC + 64;
+constexpr uint32_t OFF_ROWSQ = OFF_MISC + 64;         // fused output: [64 rows][4] partial sums of squares
+constexpr uint32_t OFF_NORMW = OFF_ROWSQ + 64 * 4 * 4;  // fused output: RMSNorm weight [128]
+constexpr uint32_t SMEM_USED = OFF_NORMW + 128 * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(64 * 64 * 4 <= 64 * AW * 4, "exact-path staging of one channel half fits the workspace");
@@ -184,6 +198,11 @@ struct Args {
   int seg_base, seg_rem;   // chunks per segment: seg_base, plus one for the first seg_rem
   float* seg_states;   // [2 n_seg - 3][H][128][128]
   const int32_t* seq_order;   // PLAN_SEQ: sequences longest first (or null: index order)
+  // MODE_FUSED: log_alpha and beta are unused; these take their place
+  const __nv_bfloat16* decay_pre;   // [T, H, 128], log alpha = logsigmoid(decay_pre)
+  const float* beta_pre;            // [T, H], beta = sigmoid(beta_pre)
+  const __nv_bfloat16* gate_pre;    // [T, H, 128], output gate = sigmoid(gate_pre)
+  const float* norm_w;              // [128] RMSNorm weight
 };
 
 struct Ctx {
@@ -261,6 +280,21 @@ __device__ __forceinline__ float rcpf(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// logsigmoid(x) = min(x, 0) - log(1 + e^{-|x|}), sigmoid(x) = 1 / (1 + e^{-x}), both on
+// the fast exp2/log2 units
+__device__ __forceinline__ float logsigmoidf_fast(float x) {
+  float l;
+  const float e = ex2f(-fabsf(x) * LOG2E);
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(l) : "f"(1.f + e));
+  return fminf(x, 0.f) - l * 0.6931471805599453f;
+}
+__device__ __forceinline__ float sigmoidf_fast(float x) { return rcpf(1.f + ex2f(-x * LOG2E)); }
+__device__ __forceinline__ uint2 ldg_nc_u2(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -295,6 +329,51 @@ __device__ __forceinline__ void tmem_block_to_tile_t(uint32_t taddr, int lane0, 
     for (int rp = 0; rp < 2; ++rp) {
       const uint32_t* w = v[hf] + 8 * rp;
       const int col = lane0 + 16 * hf + 8 * (mi & 1);       // first tile column of matrix mi
+      const int row = row0 + 8 * (2 * rp + (mi >> 1)) + (lane & 7);
+      const uint32_t addr =
+          smem_u32(tile + (col >> 6) * kb_stride) + swz128((uint32_t)row * 128u + (uint32_t)(col & 63) * 2u);
+      stmatrix_x4_trans(addr, pack_bf16(__uint_as_float(w[0]), __uint_as_float(w[1])),
+                        pack_bf16(__uint_as_float(w[2]), __uint_as_float(w[3])),
+                        pack_bf16(__uint_as_float(w[4]), __uint_as_float(w[5])),
+                        pack_bf16(__uint_as_float(w[6]), __uint_as_float(w[7])));
+    }
+}
+
+// tmem_block_to_tile_t that also sums the squares of each of the block's 32 tile rows
+// over its 32 tile columns (from the fp32 values, before rounding) and leaves the sums
+// in rowsq[row * 4 + quarter] (quarter: which 32 of the tile's 128 columns).
+__device__ __forceinline__ void tmem_block_to_tile_t_rowsq(uint32_t taddr, int lane0, int row0,
+                                                           uint8_t* tile, uint32_t kb_stride,
+                                                           int lane, float* rowsq, int quarter) {
+  uint32_t v[2][16];
+  tmem_ld16x256b_x4(taddr, v[0]);
+  tmem_ld16x256b_x4(taddr + (16u << 16), v[1]);
+  tmem_ld_wait();
+  // thread t holds columns 2(t%4), 2(t%4)+1 of every 8-row group: sum its 4 values per
+  // row, then over the 8 threads with the same t%4
+#pragma unroll
+  for (int rep = 0; rep < 4; ++rep)
+#pragma unroll
+    for (int col = 0; col < 2; ++col) {
+      float ss = 0.f;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const float a = __uint_as_float(v[hf][4 * rep + col]);
+        const float b = __uint_as_float(v[hf][4 * rep + 2 + col]);
+        ss = fmaf(a, a, fmaf(b, b, ss));
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 8);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+      if (lane < 4) rowsq[(row0 + 8 * rep + 2 * lane + col) * 4 + quarter] = ss;
+    }
+  const int mi = lane >> 3;
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+    for (int rp = 0; rp < 2; ++rp) {
+      const uint32_t* w = v[hf] + 8 * rp;
+      const int col = lane0 + 16 * hf + 8 * (mi & 1);
       const int row = row0 + 8 * (2 * rp + (mi >> 1)) + (lane & 7);
       const uint32_t addr =
           smem_u32(tile + (col >> 6) * kb_stride) + swz128((uint32_t)row * 128u + (uint32_t)(col & 63) * 2u);
@@ -465,7 +544,8 @@ __device__ __forceinline__ void issue_gram(const Ctx& x, int g) {
 // still in shared memory. Pairwise factors are evaluated one by one, one channel
 // half at a time with G staged in prep B's workspace; A goes to that workspace, P
 // to its tile, and Rk / Rq are built about the point before the chunk.
-__device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, bool sg, int c, int L,
+__device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha,
+                                          const __nv_bfloat16* decay_pre, int mode, int c, int L,
                                           uint8_t* kq, uint32_t koff, uint32_t qoff, uint8_t* ck,
                                           const float* betas) {
   const int tid = threadIdx.x;
@@ -488,9 +568,13 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, b
       const int64_t t = t0 + 8 * w + j;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
       if (t < x.eos) {
-        if (sg) {   // one gate per token and head
+        if (mode == MODE_GDN) {   // one gate per token and head
           const float a = ldg_nc_f32(log_alpha + (size_t)t * (x.rs / D) + x.h);
           v = make_float4(a, a, a, a);
+        } else if (mode == MODE_FUSED) {   // logsigmoid of the bf16 pre-activation
+          const uint2 r = ldg_nc_u2(decay_pre + (size_t)t * x.rs + x.h * D + c0);
+          v = make_float4(logsigmoidf_fast(bf_lo(r.x)), logsigmoidf_fast(bf_hi(r.x)),
+                          logsigmoidf_fast(bf_lo(r.y)), logsigmoidf_fast(bf_hi(r.y)));
         } else {
           v = ldg_nc_v4(log_alpha + (size_t)t * x.rs + x.h * D + c0);
         }
@@ -605,8 +689,9 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha, b
   return true;
 }
 
-template <bool RT, bool SG>
+template <bool RT, int MODE>
 __device__ void prep_a_role(const Ctx& x, const Args& p) {
+  constexpr bool SG = MODE == MODE_GDN, FU = MODE == MODE_FUSED;
   const int tid = threadIdx.x;
   const int w = tid >> 5, lane = tid & 31;
   const int kb = lane >> 4;                // kblock of this thread's 4 channels
@@ -619,6 +704,8 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
   // early so that its latency hides behind a whole chunk of work
   auto load_beta = [&](int cn) -> float {
     const int64_t t = x.bos + (int64_t)cn * CHUNK + tid;
+    if (FU)   // (the sigmoid is applied where the value is stored, a chunk later)
+      return (tid < 64 && t < x.eos) ? ldg_nc_f32(p.beta_pre + (size_t)t * p.n_heads + x.h) : -1e30f;
     return (tid < 64 && t < x.eos) ? ldg_nc_f32(p.beta + (size_t)t * p.n_heads + x.h) : 0.f;
   };
   float beta_next = load_beta(0);
@@ -647,6 +734,21 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
       }
       const int64_t tp = t0 + 2 * CHUNK + tid;
       if (tid < CHUNK && tp < x.eos) prefetch_l2(p.log_alpha + (size_t)tp * p.n_heads + x.h);
+    } else if (FU) {
+      // the bf16 decay pre-activation (L2-prefetched three chunks ahead), logsigmoid here
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t t = t0 + 8 * w + j;
+        uint2 r = make_uint2(0u, 0u);
+        if (t < x.eos) r = ldg_nc_u2(p.decay_pre + (size_t)t * x.rs + x.h * D + c0);
+        g2[j][0] = bf_lo(r.x); g2[j][1] = bf_hi(r.x); g2[j][2] = bf_lo(r.y); g2[j][3] = bf_hi(r.y);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const bool valid = t0 + 8 * w + j < x.eos;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) g2[j][k] = valid ? logsigmoidf_fast(g2[j][k]) : 0.f;
+      }
     } else {
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -658,7 +760,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
     }
     // (the reader of this beta slot, prep B three chunks back, finished before this
     // role got the Ck slot of chunk c-1)
-    if (tid < 64) betas[tid] = beta_next;
+    if (tid < 64) betas[tid] = FU ? sigmoidf_fast(beta_next) : beta_next;
     beta_next = load_beta(c + 1);
 
     // ---- inclusive cumsum over rows, in log2 units
@@ -689,6 +791,28 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
     }
     bool ok = wait_b(x, B_FULL + s3, (c / 3) & 1);
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
+    if (FU) {
+      // L2-normalise this warp's 8 rows of k (and q) in place: the 32 lanes hold the
+      // 128 channels of a row, 4 each; everything downstream reads the unit rows
+#pragma unroll 1
+      for (int j = 0; j < 8; ++j) {
+        const int r = 8 * w + j;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (half == 1 && lean_of<RT>(x)) break;   // (no q without output)
+          uint2* pp = reinterpret_cast<uint2*>(kq + (half ? qoff : koff) + kb * 16384 +
+                                               swz128(r * 128 + cbyte));
+          const uint2 v = *pp;
+          const float f[4] = {bf_lo(v.x), bf_hi(v.x), bf_lo(v.y), bf_hi(v.y)};
+          float ss = f[0] * f[0] + f[1] * f[1] + f[2] * f[2] + f[3] * f[3];
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+          const float inv = rsqrtf(ss + L2_EPS);
+          *pp = make_uint2(pack_bf16(f[0] * inv, f[1] * inv), pack_bf16(f[2] * inv, f[3] * inv));
+        }
+      }
+      __syncwarp();
+    }
 
     // ---- range guard: max over channels of G_0 - G_63
     bool bad = false;
@@ -737,7 +861,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
                          mul_bf16x2(kr.y, pack_bf16(f[2], f[3])));
       }
     } else {
-      ok = prep_a_exact(x, p.log_alpha, SG, c, L, kq, koff, qoff, ck, betas);
+      ok = prep_a_exact(x, p.log_alpha, p.decay_pre, MODE, c, L, kq, koff, qoff, ck, betas);
       if (!ok) break;
     }
     // per-channel scalars and the path flag of this chunk
@@ -815,9 +939,10 @@ __device__ __forceinline__ void blk_store_tb(uint8_t* tt, int a, int b, const fl
   }
 }
 
-template <bool RT, bool SG>
+template <bool RT, int MODE>
 __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
                             const CUtensorMap* map_la) {
+  constexpr bool SG = MODE == MODE_GDN;
   const int tid = threadIdx.x - PB_WARP0 * 32;
   const int q = tid >> 5, lane = tid & 31;   // q = warp within the group = TMEM lane quarter
   const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -1092,9 +1217,24 @@ __device__ __noinline__ void st_store_ragged(uint32_t lane_addr, __nv_bfloat16* 
 // state warps (12-19): the sequential pass over chunks. Thread = (TMEM lane j =
 // value column, half hh of the key channels / of the chunk rows).
 // ============================================================================
-template <bool RT>
+// (fused output) 8 bf16 outputs of one row times the row's inverse RMS, the norm
+// weight and the sigmoid of the gate pre-activation
+__device__ __forceinline__ uint4 gate_row8(uint4 o8, uint4 g8, const float* w8, float inv) {
+  const uint32_t ov[4] = {o8.x, o8.y, o8.z, o8.w}, gv[4] = {g8.x, g8.y, g8.z, g8.w};
+  uint32_t r[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float a = bf_lo(ov[i]) * inv * w8[2 * i] * sigmoidf_fast(bf_lo(gv[i]));
+    const float b = bf_hi(ov[i]) * inv * w8[2 * i + 1] * sigmoidf_fast(bf_hi(gv[i]));
+    r[i] = pack_bf16(a, b);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+template <bool RT, int MODE>
 __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v,
                            const CUtensorMap* map_o) {
+  constexpr bool FU = MODE == MODE_FUSED;
   const int tid = threadIdx.x - ST_WARP0 * 32;
   const int sw = tid >> 5, lane = tid & 31;
   const int qd = sw & 3, hh = sw >> 2;
@@ -1106,6 +1246,9 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   const int n = x.n_chunks;
 
   // ---- prologue: the fp32 state (h0, identity or zeros) and cleared output accumulators
+  float* rowsq = reinterpret_cast<float*>(x.sm + OFF_ROWSQ);
+  float* normw = reinterpret_cast<float*>(x.sm + OFF_NORMW);
+  if (FU && tid < D) normw[tid] = __ldg(p.norm_w + tid);
   st_load_state(x.tmem + TM_S + lb, x.h0, x.h0_identity, j, 64 * hh);
   if (!lean_of<RT>(x)) {
     tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
@@ -1246,7 +1389,56 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         if (alive) issue_crit<RT>(x, c);
       }
     }
-    if (c > 0 && !lean_of<RT>(x)) {
+    if (FU && c > 0 && !lean_of<RT>(x)) {
+      // ---- fused output of chunk c-1: RMSNorm over each row's 128 values, times the
+      //      weight and the sigmoid gate. (i) every warp stages its 32 x 32 block as
+      //      bf16 and leaves the fp32 row sums of squares; (ii) after the group's
+      //      barrier each thread finishes 32 values of one row from the staged tile.
+      const int co = c - 1;
+      const int64_t t0 = x.bos + (int64_t)co * CHUNK;
+      const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
+      {   // the gate rows of the next chunk into L2
+        const int64_t tn = t0 + CHUNK + (tid >> 2);
+        if (tn < x.eos) prefetch_l2(p.gate_pre + (size_t)tn * x.rs + x.h * D + 32 * (tid & 3));
+      }
+      alive = alive && wait_b(x, B_PD, co & 1);
+      if (alive) {
+        tc_fence_after();
+        const uint32_t ro = (co & 1) ? TM_OA : TM_OB;
+        tmem_block_to_tile_t_rowsq(x.tmem + ro + lb + 32 * hh, 32 * qd, 32 * hh, dt, 8192u, lane,
+                                   rowsq, qd);
+        tmem_st32_zero(x.tmem + ro + lb + 32 * hh);
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      named_bar_sync(BAR_OUT, ST_THREADS);
+      const int rr = tid >> 2, cq = tid & 3;
+      if (alive && rr < L) {
+        const float4 sq = *reinterpret_cast<const float4*>(rowsq + rr * 4);
+        const float inv = rsqrtf((sq.x + sq.y + sq.z + sq.w) * (1.f / D) + RMS_EPS);
+        const __nv_bfloat16* grow_p = p.gate_pre + (size_t)(t0 + rr) * x.rs + x.h * D;
+#pragma unroll
+        for (int sg = 0; sg < 4; ++sg) {
+          const int c8 = 32 * cq + 8 * sg;
+          uint4* tp = reinterpret_cast<uint4*>(dt + (c8 >> 6) * 8192 +
+                                               swz128((uint32_t)rr * 128u + (uint32_t)(c8 & 63) * 2u));
+          const uint4 g8 = *reinterpret_cast<const uint4*>(grow_p + c8);
+          const uint4 r8 = gate_row8(*tp, g8, normw + c8, inv);
+          if (L == CHUNK)
+            *tp = r8;
+          else   // ragged last chunk of a sequence: the valid rows go straight out
+            *reinterpret_cast<uint4*>(p.o + (size_t)(t0 + rr) * x.rs + x.h * D + c8) = r8;
+        }
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(BAR_OUT, ST_THREADS);
+      if (issuer && alive && L == CHUNK) {
+        tma_store_2d(map_o, dt, x.h * D, (int)t0);
+        tma_store_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);
+        bulk_commit_group();
+      }
+    }
+    if (!FU && c > 0 && !lean_of<RT>(x)) {
       const int co = c - 1;
       const int64_t t0 = x.bos + (int64_t)co * CHUNK;
       const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
@@ -1327,15 +1519,12 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 
 // ============================================================================
 // kernel: one CTA per (sequence, head), or per (segment, head) of a time split.
-// SG = true: Gated DeltaNet, one scalar gate per token and head (log_alpha [T, H]):
-// prep A loads 64 gate values per chunk instead of the 64 x 128 tile and evaluates
-// each row's factor once; everything downstream is the same chunk algebra.
-// RT = false (PLAN_SEQ, PLAN_OUTPUTS): every CTA writes output, and only the full
-// form of the roles is compiled. RT = true (PLAN_STATES): each CTA's flag picks the
-// lean or the full form at run time, in one body of code, so that the SMs of a TPC,
-// which share instruction caches, fetch the same code whichever CTAs they hold.
+// MODE (see the MODE_ constants): MODE_GDN reads one scalar gate per token and head and
+// prep A evaluates each row's factor once; MODE_FUSED applies the producing layer's
+// activations in prep A and the output's RMSNorm and gate in the state warps'
+// epilogue. The chunk algebra in between is the same for all three.
 // ============================================================================
-template <bool RT, bool SG>
+template <bool RT, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_la,
@@ -1416,7 +1605,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   if (threadIdx.x == 0) {
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_q);
-    if (!SG) prefetch_tensormap(&map_la);
+    if (MODE != MODE_GDN) prefetch_tensormap(&map_la);
   }
   if (warp == ST_WARP0) {
     if (lane == 0) {
@@ -1432,11 +1621,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.tmem = *tmem_slot;
 
   if (warp < PA_WARPS) {
-    prep_a_role<RT, SG>(x, args);
+    prep_a_role<RT, MODE>(x, args);
   } else if (warp < ST_WARP0) {
-    prep_b_role<RT, SG>(x, &map_k, &map_q, &map_la);
+    prep_b_role<RT, MODE>(x, &map_k, &map_q, &map_la);
   } else {
-    state_role<RT>(x, args, &map_v, &map_o);
+    state_role<RT, MODE>(x, args, &map_v, &map_o);
   }
   tc_fence_before();
   __syncthreads();

@@ -213,6 +213,67 @@ int kda_chunk_fwd_simt(const void* q, const void* k, const void* v, const float*
                        void* o, float* hT, cudaStream_t stream);
 
 /*
+ * kda_chunk_fwd_fused - kda_chunk_fwd with the producing layer's activations and the
+ * output's post-processing fused into the kernel (Kimi Linear summary, section 4 "The
+ * Kimi Linear Model Architecture"; Note, section "Other Components"; Deep-Dive,
+ * section 5.3 "Neural Parameterization"). Per head:
+ *
+ *     q = L2norm(q_pre),  k = L2norm(k_pre)          (x / sqrt(sum x^2 + 1e-12))
+ *     log alpha = logsigmoid(decay_pre)              (per channel)
+ *     beta = sigmoid(beta_pre)
+ *     (o, hT) = the KDA recurrence on (q, k, v, alpha, beta) from h0
+ *     o_out = o / sqrt(mean(o^2) + 1e-6) * norm_w * sigmoid(gate_pre)   (head-wise RMSNorm
+ *             over the 128 values of a head, then the output gate)
+ *
+ * The pages give no formula for the decay function (they call it a decay function of
+ * a low-rank projection, like those of Gated DeltaNet and Mamba); logsigmoid is the
+ * function the synthetic workloads use to draw log alpha. The short convolution and
+ * Swish that precede the normalisation are a separate call (kda_short_conv_swish).
+ * The kernel reads 256 bytes of decay per token and head instead of 512 and writes
+ * the gated output directly: no separate passes over q, k or o.
+ *
+ * Arguments (bf16 = KDA_BF16 storage; every pointer a 16-byte aligned device pointer):
+ *   q_pre, k_pre, v   [t_total, n_heads, 128] bf16 (q and k before normalisation)
+ *   decay_pre         [t_total, n_heads, 128] bf16
+ *   beta_pre          [t_total, n_heads] fp32
+ *   gate_pre          [t_total, n_heads, 128] bf16
+ *   norm_w            [128] fp32, shared by the heads
+ *   h0, cu_seqlens, n_seqs, t_total, n_heads, hT, workspace, workspace_bytes:
+ *                     as kda_chunk_fwd_ws (the same time split of one long sequence)
+ *   o                 [t_total, n_heads, 128] bf16, the gated output
+ * t_total must be 0 or at least 64 (the tensor-core path); otherwise KDA_ERR_SHAPE.
+ * Returns KDA_OK or a negative kda_status.
+ */
+int kda_chunk_fwd_fused(const void* q_pre, const void* k_pre, const void* v,
+                        const void* decay_pre, const float* beta_pre, const void* gate_pre,
+                        const float* norm_w, const float* h0, const int32_t* cu_seqlens,
+                        int32_t n_seqs, int64_t t_total, int32_t n_heads, void* o, float* hT,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * kda_short_conv_swish - the short causal depthwise convolution (4 taps) and Swish
+ * that turn the projections into q, k and v (Kimi Linear summary, section 4; Note,
+ * section "Other Components": projection, short convolution, Swish; q and k are then
+ * L2-normalised, which kda_chunk_fwd_fused does in its loader). For token t of a
+ * sequence starting at token bos and every channel c:
+ *
+ *     y_t[c] = swish(w[c][0] x_{t-3}[c] + w[c][1] x_{t-2}[c] + w[c][2] x_{t-1}[c] + w[c][3] x_t[c])
+ *
+ * with x_s = 0 for s < bos (each sequence starts without history) and swish(u) =
+ * u / (1 + e^{-u}). One call serves one tensor; q, k and v take three calls.
+ *
+ * Arguments (device pointers, 16-byte aligned):
+ *   x           [t_total, channels] bf16 (channels = n_heads * 128 for q, k, v)
+ *   w           [channels, 4] fp32, one filter per channel (tap 3 = current token)
+ *   cu_seqlens  [n_seqs + 1] int32 or NULL (one sequence), as kda_chunk_fwd
+ *   channels    a positive multiple of 8
+ *   y           [t_total, channels] bf16 output; must not be x
+ * Returns KDA_OK or a negative kda_status.
+ */
+int kda_short_conv_swish(const void* x, const float* w, const int32_t* cu_seqlens, int32_t n_seqs,
+                         int64_t t_total, int32_t channels, void* y, cudaStream_t stream);
+
+/*
  * kda_gdn_chunk_fwd - chunkwise prefill of Gated DeltaNet, the scalar-gate
  * specialisation of the same operator (Rationalist Deep-Dive, section 2.3
  * "Gated DeltaNet: The Scalar Forget"; Kimi Linear summary, section 2.2):

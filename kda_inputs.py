@@ -194,3 +194,34 @@ def make_parallel_keys(T: int, n_heads: int, qkv_dtype=torch.bfloat16, eps: floa
     h0_t = (torch.randn((1, n_heads, d, d), generator=g, device=device) * h0_std).float()
     cu = torch.tensor([0, T], dtype=torch.int32, device=device)
     return dict(q=q, k=k, v=v, log_alpha=la, beta=b, h0=h0_t, cu_seqlens=cu, lens=[T])
+
+
+def make_fused_prefill(lens, n_heads: int, x_mean: float = 3.0, h0: bool = True, seed: int = 0,
+                       device="cpu", d: int = D, h0_std: float = 0.02):
+    """Inputs of the fused entry point: the producing layer's raw outputs.
+
+    q_pre, k_pre, v ~ N(0, 1) bf16 (q and k not normalised); decay_pre ~ N(x_mean, 1)
+    bf16 (the decay pre-activation); beta_pre ~ N(0, 1) fp32; gate_pre ~ N(0, 1) bf16
+    (the output gate pre-activation); norm_w ~ U(0.5, 1.5) fp32 [d]; h0 ~ N(0, h0_std).
+    """
+    lens = [int(x) for x in lens]
+    T, N = sum(lens), len(lens)
+    g = _gen(device, seed)
+    shp = (T, n_heads, d)
+    bf = torch.bfloat16
+    out = dict(
+        q_pre=torch.randn(shp, generator=g, device=device).to(bf),
+        k_pre=torch.randn(shp, generator=g, device=device).to(bf),
+        v=torch.randn(shp, generator=g, device=device).to(bf),
+        decay_pre=(torch.randn(shp, generator=g, device=device) + x_mean).to(bf),
+        beta_pre=torch.randn((T, n_heads), generator=g, device=device).float(),
+        gate_pre=torch.randn(shp, generator=g, device=device).to(bf),
+        norm_w=(0.5 + torch.rand((d,), generator=g, device=device)).float(),
+    )
+    out["h0"] = ((torch.randn((N, n_heads, d, d), generator=g, device=device) * h0_std).float()
+                 if h0 else None)
+    cu = torch.zeros(N + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lens, dtype=torch.int64), 0).to(torch.int32)
+    out["cu_seqlens"] = cu.to(device)
+    out["lens"] = lens
+    return out

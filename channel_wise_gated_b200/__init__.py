@@ -87,6 +87,25 @@ def _prefill_args(q, k, v, gate, gate_shape_tail, beta, h0, cu_seqlens, o, hT,
     return args, (o, hT, N, T, H)
 
 
+def dplr_chunk_fwd(q, k, v, a, b, log_alpha, h0=None, cu_seqlens=None, o=None, hT=None,
+                   output_final_state: bool = True):
+    """General DPLR prefill (comparison kernel): S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} +
+    k_t v_t^T. q, k, v, a, b: [T, H, 128] bf16 or fp32 (same dtype); log_alpha: [T, H, 128]
+    fp32; h0, cu_seqlens as chunk_fwd. Returns (o, hT)."""
+    lib = _native.load()
+    for name, t in (("a", a), ("b", b)):
+        _need(t, name, q.dtype, tuple(q.shape), q.device)
+    T, H, _ = q.shape
+    dummy_beta = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    args, (o, hT, N, T, H) = _prefill_args(q, k, v, log_alpha, (D,), dummy_beta, h0, cu_seqlens,
+                                           o, hT, output_final_state)
+    q_, k_, v_, la_, _, h0_, cu_, N_, T_, H_, dt_, o_, hT_ = args
+    st = lib.kda_dplr_chunk_fwd(q_, k_, v_, _ptr(a), _ptr(b), la_, h0_, cu_, N_, T_, H_, dt_, o_,
+                                hT_, _stream_ptr(q.device))
+    _native.check(st, "kda_dplr_chunk_fwd")
+    return o, hT
+
+
 def short_conv_swish(x, w, cu_seqlens=None, y=None):
     """Causal 4-tap depthwise convolution + Swish over tokens, restarted per sequence.
 

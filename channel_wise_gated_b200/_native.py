@@ -42,6 +42,8 @@ SIGNATURES = {
     "kda_chunk_fwd_static": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
     "kda_chunk_fwd_fused": [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, _P, _P, _P,
                             ctypes.c_size_t, _P],
+    "kda_dplr_chunk_fwd": [_P, _P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P,
+                           _P],
     "kda_short_conv_swish": [_P, _P, _P, _I32, _I64, _I32, _P, _P],
     "kda_gdn_chunk_fwd": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P],
     "kda_gdn_chunk_fwd_ws": [_P, _P, _P, _P, _P, _P, _P, _I32, _I64, _I32, ctypes.c_int, _P, _P, _P,

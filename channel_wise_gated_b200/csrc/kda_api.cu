@@ -15,6 +15,7 @@
 #include "kda_common.cuh"
 #include "kda_conv.cuh"
 #include "kda_decode.cuh"
+#include "kda_dplr_simt.cuh"
 #include "kda_segment.cuh"
 
 // Scratch of kda_chunk_fwd_static, for callers that cannot allocate device memory:
@@ -484,6 +485,38 @@ int kda_chunk_fwd_fused(const void* q_pre, const void* k_pre, const void* v,
   return launch_chunk_tc<kda::tc::MODE_FUSED>(q_pre, k_pre, v, nullptr, nullptr, h0, cu_seqlens,
                                               n_seqs, t_total, n_heads, o, hT, n_seg,
                                               static_cast<float*>(workspace), order, &fu, stream);
+}
+
+int kda_dplr_chunk_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                       const float* log_alpha, const float* h0, const int32_t* cu_seqlens,
+                       int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                       void* o, float* hT, cudaStream_t stream) {
+  int st = validate_chunk_args(q, k, v, log_alpha, log_alpha, h0, cu_seqlens, n_seqs, t_total,
+                               n_heads, qkv_dtype, o, hT);
+  if (st != KDA_OK) return st;
+  if (t_total > 0 && (!a || !b)) return KDA_ERR_NULL;
+  if ((a && !aligned16(a)) || (b && !aligned16(b))) return KDA_ERR_ALIGN;
+  const size_t smem = sizeof(kda::DplrSmem);
+  dim3 grid((unsigned)(n_seqs * n_heads), kda::D / kda::DPLR_DV);
+  if (qkv_dtype == KDA_F32) {
+    if (cudaFuncSetAttribute(kda::kda_dplr_simt_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    kda::kda_dplr_simt_kernel<float><<<grid, kda::DPLR_THREADS, smem, stream>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<const float*>(a), static_cast<const float*>(b), log_alpha, h0, cu_seqlens,
+        n_seqs, t_total, n_heads, static_cast<float*>(o), hT);
+  } else {
+    using bf = __nv_bfloat16;
+    if (cudaFuncSetAttribute(kda::kda_dplr_simt_kernel<bf>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    kda::kda_dplr_simt_kernel<bf><<<grid, kda::DPLR_THREADS, smem, stream>>>(
+        static_cast<const bf*>(q), static_cast<const bf*>(k), static_cast<const bf*>(v),
+        static_cast<const bf*>(a), static_cast<const bf*>(b), log_alpha, h0, cu_seqlens, n_seqs,
+        t_total, n_heads, static_cast<bf*>(o), hT);
+  }
+  return launch_status();
 }
 
 int kda_short_conv_swish(const void* x, const float* w, const int32_t* cu_seqlens, int32_t n_seqs,

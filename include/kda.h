@@ -251,6 +251,30 @@ int kda_chunk_fwd_fused(const void* q_pre, const void* k_pre, const void* v,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * kda_dplr_chunk_fwd - chunkwise prefill of the general DPLR recurrence, the operator
+ * the pages compare KDA's kernel against (Rationalist Deep-Dive, section 3.2 "DPLR
+ * Structure"; Kimi Linear summary, sections 3.2 "Efficiency Analysis" and 6.2
+ * "Relation to DPLR"):
+ *
+ *     S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} + k_t v_t^T,   o_t = S_t^T q_t
+ *
+ * with free low-rank factors a_t, b_t (KDA ties them, a = beta k and b = k * alpha,
+ * which reduces the chunk form's four decayed Gram matrices to two). This is a
+ * comparison kernel: fp32 CUDA-core arithmetic with exact pairwise decay factors, in
+ * the style of kda_chunk_fwd_simt, so the two chunk algorithms can be timed on the
+ * same footing.
+ *
+ * Arguments: as kda_chunk_fwd (q, k, v, h0, cu_seqlens, sizes, dtype, o, hT), plus
+ *   a, b   [t_total, n_heads, 128], dtype qkv_dtype
+ * log_alpha [t_total, n_heads, 128] fp32 as for KDA. Returns KDA_OK or a negative
+ * kda_status.
+ */
+int kda_dplr_chunk_fwd(const void* q, const void* k, const void* v, const void* a, const void* b,
+                       const float* log_alpha, const float* h0, const int32_t* cu_seqlens,
+                       int32_t n_seqs, int64_t t_total, int32_t n_heads, kda_dtype qkv_dtype,
+                       void* o, float* hT, cudaStream_t stream);
+
+/*
  * kda_short_conv_swish - the short causal depthwise convolution (4 taps) and Swish
  * that turn the projections into q, k and v (Kimi Linear summary, section 4; Note,
  * section "Other Components": projection, short convolution, Swish; q and k are then

@@ -225,3 +225,21 @@ def make_fused_prefill(lens, n_heads: int, x_mean: float = 3.0, h0: bool = True,
     out["cu_seqlens"] = cu.to(device)
     out["lens"] = lens
     return out
+
+
+def make_dplr_prefill(lens, n_heads: int, qkv_dtype=torch.bfloat16, x_mean: float = 3.0,
+                      h0: bool = True, seed: int = 0, device="cpu", d: int = D,
+                      h0_std: float = 0.02):
+    """Inputs of the general DPLR recurrence: those of make_prefill plus free low-rank
+    factors a = beta u and b = w * alpha, with u and w unit vectors drawn independently
+    of k (KDA would take u = w = k). Returns make_prefill's dict plus a and b."""
+    inp = make_prefill(lens, n_heads, qkv_dtype, torch.float32, x_mean, h0, seed, device,
+                       d=d, h0_std=h0_std)
+    g = _gen(device, seed + 7777)
+    T = sum(int(x) for x in lens)
+    shp = (T, n_heads, d)
+    u = _unit_rows(torch.randn(shp, generator=g, device=device))
+    w = _unit_rows(torch.randn(shp, generator=g, device=device))
+    inp["a"] = (inp["beta"][:, :, None] * u).to(qkv_dtype)
+    inp["b"] = (w * torch.exp(inp["log_alpha"])).to(qkv_dtype)
+    return inp

@@ -65,3 +65,41 @@ def chunk_forward(q, k, v, beta, log_alpha, S0=None, chunk: int = 64):
         gC = G[-1]
         S = np.exp(gC)[:, None] * S + (K * np.exp(gC[None, :] - G)).T @ Delta
     return o, S
+
+
+def dplr_chunked(q, k, v, a, b, log_alpha, S0, C=64):
+    """General DPLR, S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} + k_t v_t^T, by chunks (fp64,
+    one head), derived from the recurrence: within a chunk with inclusive cumulative log
+    decay G (G_{-1} = 0) and correction rows u_r = b_r^T S_{r-1},
+        S_r = Diag(e^{G_r}) S_0 + sum_{i<=r} Diag(e^{G_r - G_i}) (k_i v_i^T - a_i u_i^T),
+    so with the decayed Grams (i < r)  Mbk_ri = b_r . (e^{G_{r-1} - G_i} k_i),
+    Mba_ri = b_r . (e^{G_{r-1} - G_i} a_i) and (i <= r)  Mqk_ri = q_r . (e^{G_r - G_i} k_i),
+    Mqa_ri = q_r . (e^{G_r - G_i} a_i):
+        (I + Mba) U = (B * e^{G_prev}) S_0 + Mbk V
+        O = (Q * e^G) S_0 + Mqk V - Mqa U
+        S_C = Diag(e^{G_C}) S_0 + (K * e^{G_C - G})^T V - (A * e^{G_C - G})^T U.
+    Four decayed Grams where KDA's tied factors need two."""
+    T, dk = q.shape
+    S = np.array(S0, dtype=np.float64)
+    o = np.zeros((T, v.shape[1]))
+    for t0 in range(0, T, C):
+        sl = slice(t0, min(T, t0 + C))
+        Q, K, V, A, B = q[sl], k[sl], v[sl], a[sl], b[sl]
+        G = np.cumsum(log_alpha[sl], axis=0)
+        Gp = np.vstack([np.zeros((1, dk)), G[:-1]])
+        L = Q.shape[0]
+        Mbk = np.zeros((L, L)); Mba = np.zeros((L, L)); Mqk = np.zeros((L, L)); Mqa = np.zeros((L, L))
+        for r in range(L):
+            for i in range(r + 1):
+                ec = np.exp(G[r] - G[i])
+                Mqk[r, i] = Q[r] @ (ec * K[i])
+                Mqa[r, i] = Q[r] @ (ec * A[i])
+                if i < r:
+                    ep = np.exp(Gp[r] - G[i])
+                    Mbk[r, i] = B[r] @ (ep * K[i])
+                    Mba[r, i] = B[r] @ (ep * A[i])
+        U = np.linalg.solve(np.eye(L) + Mba, (B * np.exp(Gp)) @ S + Mbk @ V)
+        o[sl] = (Q * np.exp(G)) @ S + Mqk @ V - Mqa @ U
+        F = np.exp(G[-1] - G)
+        S = np.exp(G[-1])[:, None] * S + (K * F).T @ V - (A * F).T @ U
+    return o, S

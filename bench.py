@@ -86,6 +86,22 @@ def _profiled_traffic(split: bool, token_heads: int):
     return float(mb.group(1)) * token_heads
 
 
+def _profiled_metric(name: str):
+    """A figure recorded with the ncu capture summarised in
+    profiles/kda_chunk_tc_prefill4k_full.md, or None when the kernel sources changed
+    since that capture."""
+    import re
+    path = os.path.join(ROOT, "profiles", "kda_chunk_tc_prefill4k_full.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    mh = re.search(r"^source_hash: ([0-9a-f]+)$", txt, re.M)
+    mv = re.search(rf"^{name}: ([0-9.]+)$", txt, re.M)
+    if not mh or not mv or mh.group(1) != _source_hash():
+        return None
+    return float(mv.group(1))
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
@@ -350,6 +366,131 @@ def time_decode_tokens(kda, pool, state, calls, warmup, stream):
     return a.elapsed_time(b)
 
 
+def _time_calls(fn, reps, warmup, stream):
+    """Average CUDA-event time of `reps` back-to-back calls on `stream`, after warm-up."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def _frac(nbytes, ms, peak_gbs):
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"GBps": gbs, "frac": gbs / peak_gbs, "frac_nominal_8tbs": gbs / 8000.0,
+            "algorithmic_bytes": nbytes}
+
+
+def run_extras(kda, hbm_peak, stream, headline):
+    """The other entry points and workloads, each timed on its own (N = 1): the
+    contract's single-pass call at the headline size, the T=4096 and packed-batch
+    prefills, the Gated DeltaNet and fused-layer variants at the headline size, the
+    short convolution, and the general-DPLR comparison (16 heads, batch 1). Inputs are
+    drawn on the device before each entry's timed region and larger than L2 where the
+    entry is an HBM-bound pass."""
+    ex = {}
+    D_ = D
+    # (1) the contract's entry point (single pass, no workspace) on the headline input
+    inp = headline
+    T, H = inp["q"].shape[0], inp["q"].shape[1]
+    ms = _time_calls(lambda: kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"],
+                                           inp["beta"], o=inp["o"], hT=inp["hT"],
+                                           kernel="single"), 2, 1, stream)
+    nbytes = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    ex["contract_single_pass"] = {"entry": "kda_chunk_fwd", "workload": "longctx_bf16_T1048576_H32",
+                                  "ms": ms, "tokens_per_s": T / (ms / 1e3),
+                                  **_frac(nbytes, ms, hbm_peak)}
+    # (2) the smaller prefill workloads, through the workspace entry point
+    for key, idx in (("prefill4k", 1), ("varlen16", 2)):
+        cfg = kda_inputs.PREFILL_CONFIGS[idx]
+        lens = kda_inputs.config_lengths(cfg)
+        x = kda_inputs.make_prefill(lens, cfg.n_heads, cfg.qkv_dtype, torch.float32, cfg.x_mean,
+                                    cfg.h0, cfg.seed, "cuda")
+        cu = None if len(lens) == 1 else x["cu_seqlens"]
+        ms = _time_calls(lambda: kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                               h0=x["h0"], cu_seqlens=cu), 20, 3, stream)
+        Tt, N = sum(lens), len(lens)
+        nbytes = Tt * cfg.n_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * N * cfg.n_heads * STATE_BYTES
+        ex[key] = {"entry": "kda_chunk_fwd_ws", "workload": cfg.name, "ms": ms,
+                   "tokens_per_s": Tt / (ms / 1e3), **_frac(nbytes, ms, hbm_peak)}
+        del x
+    torch.cuda.empty_cache()
+    return ex
+
+
+def run_extras_large(kda, hbm_peak, stream, ex):
+    """Entries whose inputs are as large as the headline's (run after it is freed)."""
+    cfg = kda_inputs.PREFILL_CONFIGS[3]
+    T, H = cfg.lens[0], cfg.n_heads
+    # (3) Gated DeltaNet: one gate per token and head (4 B instead of 512)
+    x = kda_inputs.make_prefill([T], H, cfg.qkv_dtype, torch.float32, cfg.x_mean, cfg.h0,
+                                cfg.seed, "cuda", scalar_gate=True)
+    o = torch.empty_like(x["q"])
+    hT = torch.empty((1, H, D, D), dtype=torch.float32, device="cuda")
+    ms = _time_calls(lambda: kda.gdn_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                               o=o, hT=hT), 5, 3, stream)
+    per_th = 3 * 2 * D + 4 + 4 + 2 * D
+    ex["gdn_scalar_gate"] = {"entry": "kda_gdn_chunk_fwd_ws", "workload": f"{cfg.name}_scalar_gate",
+                             "ms": ms, "tokens_per_s": T / (ms / 1e3),
+                             "bytes_per_token_head": per_th,
+                             **_frac(T * H * per_th + H * STATE_BYTES, ms, hbm_peak)}
+    del x, o, hT
+    torch.cuda.empty_cache()
+    # (4) the fused layer path: L2 norm, logsigmoid, sigmoid in the loader, RMSNorm and
+    #     gate in the epilogue (bf16 decay 256 B, gate 256 B per token-head)
+    x = kda_inputs.make_fused_prefill([T], H, x_mean=cfg.x_mean, h0=False, seed=cfg.seed,
+                                      device="cuda")
+    o = torch.empty_like(x["q_pre"])
+    hT = torch.empty((1, H, D, D), dtype=torch.float32, device="cuda")
+    ms = _time_calls(lambda: kda.chunk_fwd_fused(x["q_pre"], x["k_pre"], x["v"], x["decay_pre"],
+                                                 x["beta_pre"], x["gate_pre"], x["norm_w"],
+                                                 o=o, hT=hT), 5, 3, stream)
+    per_th = 3 * 2 * D + 2 * D + 4 + 2 * D + 2 * D   # q k v, decay, beta, gate, o
+    ex["fused_layer"] = {"entry": "kda_chunk_fwd_fused", "workload": f"{cfg.name}_fused",
+                         "ms": ms, "tokens_per_s": T / (ms / 1e3),
+                         "bytes_per_token_head": per_th,
+                         "unfused_passes_bytes_per_token_head": (
+                             PREFILL_BYTES_PER_TOKEN_HEAD   # the operator itself (fp32 log alpha)
+                             + 4 * 2 * D                    # L2 norm of q, k: read + write
+                             + 2 * D + 4 * D                # decay activation: read bf16, write fp32
+                             + 3 * 2 * D),                  # RMSNorm + gate: read o, gate; write
+                         **_frac(T * H * per_th + H * STATE_BYTES, ms, hbm_peak)}
+    # (5) the short convolution + Swish of one of q, k, v at the same size
+    C = H * D
+    wc = (torch.randn((C, 4), device="cuda") * 0.5).float()
+    xin = x["q_pre"].reshape(T, C)
+    y = torch.empty_like(xin)
+    ms = _time_calls(lambda: kda.short_conv_swish(xin, wc, y=y), 5, 3, stream)
+    ex["short_conv_swish"] = {"entry": "kda_short_conv_swish", "workload": f"T{T}_C{C}_bf16",
+                              "ms": ms, "tokens_per_s": T / (ms / 1e3),
+                              **_frac(T * C * 2 * 2, ms, hbm_peak)}
+    del x, o, hT, xin, y
+    torch.cuda.empty_cache()
+    # (6) general DPLR against KDA, the same CUDA-core style, 16 heads, batch 1
+    rows = []
+    for Tc in (2048, 8192, 65536):
+        x = kda_inputs.make_dplr_prefill([Tc], 16, torch.bfloat16, seed=1, device="cuda")
+        t_k = _time_calls(lambda: kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                                                h0=x["h0"], kernel="simt"), 2, 1, stream)
+        t_d = _time_calls(lambda: kda.dplr_chunk_fwd(x["q"], x["k"], x["v"], x["a"], x["b"],
+                                                     x["log_alpha"], h0=x["h0"]), 2, 1, stream)
+        t_tc = _time_calls(lambda: kda.chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"],
+                                                 x["beta"], h0=x["h0"]), 5, 2, stream)
+        rows.append({"T": Tc, "H": 16, "kda_cuda_core_ms": t_k, "dplr_cuda_core_ms": t_d,
+                     "dplr_over_kda": t_d / t_k, "kda_tensor_core_ms": t_tc})
+        del x
+    torch.cuda.empty_cache()
+    ex["dplr_comparison"] = {"entries": ["kda_chunk_fwd_simt", "kda_dplr_chunk_fwd",
+                                         "kda_chunk_fwd_ws"], "rows": rows}
+    return ex
+
+
 def time_e2e(kda, inp, steps, stream):
     """Public API with host buffers: H2D of the step's inputs from pinned memory,
     the prefill, and D2H of its outputs (o and the final state), every step."""
@@ -397,6 +538,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other entry points' entries (timed after the headline)")
     ap.add_argument("--workload", default="longctx",
                     choices=sorted(WORKLOADS),
                     help="prefill workload (the headline is longctx; prefill4k is the small "
@@ -474,6 +617,14 @@ def main():
                "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
+    extras = None
+    if ws == 1 and not args.no_extras and args.workload == "longctx":
+        extras = run_extras(kda, hbm_peak, stream, inp)
+    del inp
+    torch.cuda.empty_cache()
+    if extras is not None:
+        extras = run_extras_large(kda, hbm_peak, stream, extras)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, desc, threads, _, _ = _oracle_sample_rate(3, 12.0)
@@ -492,6 +643,8 @@ def main():
                        "parallelism": f"replicas x{ws}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                          "frac": achieved / hbm_peak,
+                         "frac_nominal_8tbs": achieved / 8000.0,
+                         "tensor_pipe_pct": _profiled_metric("tensor_pipe_active_pct"),
                          "traffic": _profiled_traffic(split, T * H),
                          "traffic_note": ("DRAM bytes per call from the ncu capture of "
                                           "profiles/kda_chunk_tc_prefill4k_full.md, scaled by "
@@ -513,6 +666,7 @@ def main():
                                     "algorithmic_bytes_per_step": chains * DECODE_BYTES_PER_CHAIN},
                        "gpu_launches": args.decode_steps,
                        "l2": "state 512 MiB > L2"},
+            "extras": extras if extras is not None else "skipped (N > 1 or --no-extras)",
             "decode_tokens": {"workload": f"{dcfg.name}_t{t_dec}", "calls": dt_calls,
                               "tokens_per_call": t_dec,
                               "us_per_call": dt_ms / dt_calls * 1e3,

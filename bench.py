@@ -71,19 +71,19 @@ def _source_hash() -> str:
 
 
 def _profiled_traffic(split: bool, token_heads: int):
-    """DRAM bytes per prefill call from the committed ncu summary, scaled to this
-    workload by its token-heads, or None when the kernel sources changed since the
-    capture (or the capture does not describe this kind of call)."""
+    """DRAM bytes of one long-context prefill call from the committed one-pass ncu capture
+    (profiles/kda_chunk_tc_longctx_dram.md), or None when the kernel sources changed since
+    that capture or the call is not the one it describes."""
     import re
-    path = os.path.join(ROOT, "profiles", "kda_chunk_tc_prefill4k_full.md")
-    if not split or not os.path.exists(path):
+    path = os.path.join(ROOT, "profiles", "kda_chunk_tc_longctx_dram.md")
+    if not split or token_heads != 32 * 1048576 or not os.path.exists(path):
         return None
     txt = open(path).read()
     mh = re.search(r"^source_hash: ([0-9a-f]+)$", txt, re.M)
-    mb = re.search(r"^split_call_dram_bytes_per_token_head: ([0-9.]+)$", txt, re.M)
+    mb = re.search(r"^longctx_call_dram_bytes: ([0-9.]+)$", txt, re.M)
     if not mh or not mb or mh.group(1) != _source_hash():
         return None
-    return float(mb.group(1)) * token_heads
+    return float(mb.group(1))
 
 
 def _profiled_metric(name: str):
@@ -646,9 +646,9 @@ def main():
                          "frac_nominal_8tbs": achieved / 8000.0,
                          "tensor_pipe_pct": _profiled_metric("tensor_pipe_active_pct"),
                          "traffic": _profiled_traffic(split, T * H),
-                         "traffic_note": ("DRAM bytes per call from the ncu capture of "
-                                          "profiles/kda_chunk_tc_prefill4k_full.md, scaled by "
-                                          "token-heads; null if the kernel changed since"),
+                         "traffic_note": ("DRAM bytes of one call from the one-pass ncu capture "
+                                          "of the same call, profiles/kda_chunk_tc_longctx_dram.md;"
+                                          " null if the kernel changed since"),
                          "peak_kind": peak_kind,
                          "kernel": "kda_chunk_tc_kernel",
                          "unit_of_work": ("one prefill call (state pass + segment scan + "

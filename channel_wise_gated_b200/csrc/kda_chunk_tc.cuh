@@ -289,6 +289,12 @@ __device__ __forceinline__ float logsigmoidf_fast(float x) {
   return fminf(x, 0.f) - l * 0.6931471805599453f;
 }
 __device__ __forceinline__ float sigmoidf_fast(float x) { return rcpf(1.f + ex2f(-x * LOG2E)); }
+__device__ __forceinline__ uint4 ldg_nc_u4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
 __device__ __forceinline__ uint2 ldg_nc_u2(const void* p) {
   uint2 v;
   asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
@@ -793,24 +799,40 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
     if (FU) {
       // L2-normalise this warp's 8 rows of k (and q) in place: the 32 lanes hold the
-      // 128 channels of a row, 4 each; everything downstream reads the unit rows
-#pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        const int r = 8 * w + j;
+      // 128 channels of a row, 4 each. All 16 row sums first, then their butterflies
+      // side by side (independent shuffle chains), then the rescaled rows written back;
+      // everything downstream reads the unit rows.
+      const bool do_q = !lean_of<RT>(x);
+      float ss[2][8];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if (half == 1 && lean_of<RT>(x)) break;   // (no q without output)
-          uint2* pp = reinterpret_cast<uint2*>(kq + (half ? qoff : koff) + kb * 16384 +
-                                               swz128(r * 128 + cbyte));
-          const uint2 v = *pp;
-          const float f[4] = {bf_lo(v.x), bf_hi(v.x), bf_lo(v.y), bf_hi(v.y)};
-          float ss = f[0] * f[0] + f[1] * f[1] + f[2] * f[2] + f[3] * f[3];
+      for (int half = 0; half < 2; ++half)
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-          const float inv = rsqrtf(ss + L2_EPS);
-          *pp = make_uint2(pack_bf16(f[0] * inv, f[1] * inv), pack_bf16(f[2] * inv, f[3] * inv));
+        for (int j = 0; j < 8; ++j) {
+          ss[half][j] = 0.f;
+          if (half == 1 && !do_q) continue;
+          const uint2 v = *reinterpret_cast<const uint2*>(kq + (half ? qoff : koff) + kb * 16384 +
+                                                          swz128((8 * w + j) * 128 + cbyte));
+          const float f0 = bf_lo(v.x), f1 = bf_hi(v.x), f2 = bf_lo(v.y), f3 = bf_hi(v.y);
+          ss[half][j] = f0 * f0 + f1 * f1 + f2 * f2 + f3 * f3;
         }
-      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int half = 0; half < 2; ++half)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss[half][j] += __shfl_xor_sync(0xffffffffu, ss[half][j], off);
+#pragma unroll
+      for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (half == 1 && !do_q) continue;
+          uint2* pp = reinterpret_cast<uint2*>(kq + (half ? qoff : koff) + kb * 16384 +
+                                               swz128((8 * w + j) * 128 + cbyte));
+          const uint2 v = *pp;
+          const float inv = rsqrtf(ss[half][j] + L2_EPS);
+          *pp = make_uint2(pack_bf16(bf_lo(v.x) * inv, bf_hi(v.x) * inv),
+                           pack_bf16(bf_lo(v.y) * inv, bf_hi(v.y) * inv));
+        }
       __syncwarp();
     }
 
@@ -1401,6 +1423,16 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         const int64_t tn = t0 + CHUNK + (tid >> 2);
         if (tn < x.eos) prefetch_l2(p.gate_pre + (size_t)tn * x.rs + x.h * D + 32 * (tid & 3));
       }
+      // this thread's 32 gate values of the chunk (row rr, channels 32 cq ..), in flight
+      // while the block is staged
+      const int rr = tid >> 2, cq = tid & 3;
+      uint4 g8[4];
+      {
+        const __nv_bfloat16* gp = p.gate_pre + (size_t)(t0 + rr) * x.rs + x.h * D + 32 * cq;
+#pragma unroll
+        for (int sg = 0; sg < 4; ++sg)
+          g8[sg] = rr < L ? ldg_nc_u4(gp + 8 * sg) : make_uint4(0u, 0u, 0u, 0u);
+      }
       alive = alive && wait_b(x, B_PD, co & 1);
       if (alive) {
         tc_fence_after();
@@ -1412,18 +1444,15 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         tc_fence_before();
       }
       named_bar_sync(BAR_OUT, ST_THREADS);
-      const int rr = tid >> 2, cq = tid & 3;
       if (alive && rr < L) {
         const float4 sq = *reinterpret_cast<const float4*>(rowsq + rr * 4);
         const float inv = rsqrtf((sq.x + sq.y + sq.z + sq.w) * (1.f / D) + RMS_EPS);
-        const __nv_bfloat16* grow_p = p.gate_pre + (size_t)(t0 + rr) * x.rs + x.h * D;
 #pragma unroll
         for (int sg = 0; sg < 4; ++sg) {
           const int c8 = 32 * cq + 8 * sg;
           uint4* tp = reinterpret_cast<uint4*>(dt + (c8 >> 6) * 8192 +
                                                swz128((uint32_t)rr * 128u + (uint32_t)(c8 & 63) * 2u));
-          const uint4 g8 = *reinterpret_cast<const uint4*>(grow_p + c8);
-          const uint4 r8 = gate_row8(*tp, g8, normw + c8, inv);
+          const uint4 r8 = gate_row8(*tp, g8[sg], normw + c8, inv);
           if (L == CHUNK)
             *tp = r8;
           else   // ragged last chunk of a sequence: the valid rows go straight out

@@ -116,7 +116,6 @@ kda_dplr_simt_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k, const T
       for (int r = warp; r < CHUNK; r += STRIDE) {
         const float* Br = &sm.B[r * DPLR_LDH];
         const float* Qr = &sm.Q[r * DPLR_LDH];
-        const float* Gr = &sm.G[r * DPLR_LDH];
         const float* Ar = &sm.Al[r * DPLR_LDH];
         const float* Gp = r > 0 ? &sm.G[(r - 1) * DPLR_LDH] : nullptr;
 #pragma unroll

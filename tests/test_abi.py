@@ -57,21 +57,25 @@ def test_every_exported_entry_point_is_declared(lib):
     assert set(exported) <= set(declared_functions()), set(exported) - set(declared_functions())
 
 
-def test_profile_summary_is_machine_readable():
-    """bench.py reads the DRAM traffic per token-head and the kernel-source hash it was
-    taken with from the committed ncu summary; both must parse."""
+def test_profile_summaries_are_machine_readable():
+    """bench.py reads the long-context call's DRAM bytes and the tensor-pipe activity,
+    each with the kernel-source hash it was taken with, from the committed ncu
+    summaries; all must parse and be plausible."""
     import importlib.util
     spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
     bench_mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(bench_mod)
     for f in bench_mod.CHUNK_KERNEL_SOURCES:
         assert os.path.exists(os.path.join(ROOT, "channel_wise_gated_b200", "csrc", f)), f
-    text = open(os.path.join(ROOT, "profiles", "kda_chunk_tc_prefill4k_full.md")).read()
-    mh = re.search(r"^source_hash: ([0-9a-f]{16})$", text, re.M)
-    mb = re.search(r"^split_call_dram_bytes_per_token_head: ([0-9.]+)$", text, re.M)
-    assert mh and mb
-    # at least the algorithmic 1,540 B per token-head, at most a few times it
-    assert 1540 <= float(mb.group(1)) <= 8 * 1540
+    dram = open(os.path.join(ROOT, "profiles", "kda_chunk_tc_longctx_dram.md")).read()
+    assert re.search(r"^source_hash: ([0-9a-f]{16})$", dram, re.M)
+    mb = re.search(r"^longctx_call_dram_bytes: ([0-9.]+)$", dram, re.M)
+    # at least the algorithmic 51.68 GB of the call, at most a few times it
+    assert mb and 51.68e9 <= float(mb.group(1)) <= 4 * 51.68e9
+    full = open(os.path.join(ROOT, "profiles", "kda_chunk_tc_prefill4k_full.md")).read()
+    assert re.search(r"^source_hash: ([0-9a-f]{16})$", full, re.M)
+    mt = re.search(r"^tensor_pipe_active_pct: ([0-9.]+)$", full, re.M)
+    assert mt and 0.0 < float(mt.group(1)) <= 100.0
     assert re.fullmatch(r"[0-9a-f]{16}", bench_mod._source_hash())
 
 

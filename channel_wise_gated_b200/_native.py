@@ -51,6 +51,8 @@ SIGNATURES = {
     "kda_decode_step": [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, ctypes.c_int, ctypes.c_int, _P],
     "kda_decode_tokens": [_P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, ctypes.c_int, ctypes.c_int,
                           _P],
+    "kda_testing_chunk_fwd_stall": [_P, _P, _P, _P, _P, _P, _I64, _I32, _P, _P, _I32, ctypes.c_uint32,
+                                    _P],
     "kda_device_status": [_P],
     "kda_status_string": [ctypes.c_int],
 }

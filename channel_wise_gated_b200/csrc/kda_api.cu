@@ -194,7 +194,8 @@ template <int MODE>
 int launch_chunk_tc(const void* q, const void* k, const void* v, const float* log_alpha,
                     const float* beta, const float* h0, const int32_t* cu_seqlens, int32_t n_seqs,
                     int64_t t_total, int32_t n_heads, void* o, float* hT, int n_seg,
-                    float* seg_states, int32_t* seq_order, const FusedIO* fu, cudaStream_t stream) {
+                    float* seg_states, int32_t* seq_order, const FusedIO* fu, cudaStream_t stream,
+                    uint64_t wait_ns = 0, int debug_skip_tb = -1) {
   using namespace kda::tc;
   const uint64_t cols = (uint64_t)n_heads * kda::D;
   const uint64_t rows = (uint64_t)t_total;
@@ -242,6 +243,8 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
   a.beta_pre = fu ? fu->beta_pre : nullptr;
   a.gate_pre = fu ? static_cast<const __nv_bfloat16*>(fu->gate_pre) : nullptr;
   a.norm_w = fu ? fu->norm_w : nullptr;
+  a.wait_ns = wait_ns;
+  a.debug_skip_tb = debug_skip_tb;
   if (seq_order != nullptr && cu_seqlens != nullptr && n_seqs > 1) {
     const unsigned blocks = (unsigned)((n_seqs + kda::seg::ORDER_THREADS - 1) / kda::seg::ORDER_THREADS);
     kda::seg::kda_seq_order_kernel<<<blocks, kda::seg::ORDER_THREADS, 0, stream>>>(
@@ -627,6 +630,19 @@ int kda_decode_tokens(const void* q, const void* k, const void* v, const void* l
                                                       n_tokens, n_heads, stream);
   return launch_decode_tokens<float, float>(q, k, v, log_alpha, beta, state, o, n_seqs, n_tokens,
                                             n_heads, stream);
+}
+
+int kda_testing_chunk_fwd_stall(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, const float* h0,
+                                int64_t t_total, int32_t n_heads, void* o, float* hT,
+                                int32_t skip_chunk, uint32_t wait_us, cudaStream_t stream) {
+  int st = validate_chunk_args(q, k, v, log_alpha, beta, h0, nullptr, 1, t_total, n_heads, KDA_BF16,
+                               o, hT);
+  if (st != KDA_OK) return st;
+  if (!use_tc(nullptr, 1, t_total, n_heads, KDA_BF16) || wait_us == 0) return KDA_ERR_SHAPE;
+  return launch_chunk_tc<kda::tc::MODE_KDA>(q, k, v, log_alpha, beta, h0, nullptr, 1, t_total,
+                                            n_heads, o, hT, 0, nullptr, nullptr, nullptr, stream,
+                                            (uint64_t)wait_us * 1000ull, skip_chunk);
 }
 
 int kda_device_status(cudaStream_t stream) {

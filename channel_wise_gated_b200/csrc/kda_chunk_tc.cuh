@@ -74,7 +74,7 @@ constexpr uint32_t BAR_PA = 1, BAR_PB = 2, BAR_ST = 3;   // named barriers (0 is
 constexpr uint32_t BAR_OUT = 4;   // state warps: output tile staged (arrive), then stored
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float GUARD_LOG2 = 60.0f * 1.4426950408889634f;
-constexpr uint64_t WAIT_NS = 2000000000ull;
+constexpr uint64_t WAIT_NS = 2000000000ull;   // bound of every wait (unless a test sets its own)
 
 // What the kernel reads and writes around the recurrence:
 //   MODE_KDA    q, k (unit length), v, log_alpha [T, H, 128] fp32, beta [T, H] fp32 -> o
@@ -110,7 +110,8 @@ constexpr uint32_t OFF_GROW = OFF_WSUM + 8 * 128 * 4; // [2][128] G of rows 0 an
 constexpr uint32_t OFF_XFLAG = OFF_GROW + 2 * 128 * 4; // [3] exact-path flag per slot
 constexpr uint32_t OFF_BAR = OFF_XFLAG + 16;
 constexpr int NBARS = 32;
-constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr uint32_t OFF_MISC = OFF_BAR + NBARS * 8;   // abort word, TMEM address, wait bound, test hook
+constexpr uint32_t MISC_TMEM = 8, MISC_WAIT_NS = 16, MISC_SKIP_TB = 24;   // byte offsets in MISC
 constexpr uint32_t OFF_ROWSQ = OFF_MISC + 64;         // fused output: [64 rows][4] partial sums of squares
 constexpr uint32_t OFF_NORMW = OFF_ROWSQ + 64 * 4 * 4;  // fused output: RMSNorm weight [128]
 constexpr uint32_t SMEM_USED = OFF_NORMW + 128 * 4;
@@ -203,6 +204,10 @@ struct Args {
   const float* beta_pre;            // [T, H], beta = sigmoid(beta_pre)
   const __nv_bfloat16* gate_pre;    // [T, H, 128], output gate = sigmoid(gate_pre)
   const float* norm_w;              // [128] RMSNorm weight
+  // testing only (kda_testing_chunk_fwd_stall): the bound of every wait, and one chunk
+  // whose "T*beta ready" arrive prep B leaves out (-1: none)
+  uint64_t wait_ns;
+  int debug_skip_tb;
 };
 
 struct Ctx {
@@ -236,12 +241,15 @@ constexpr int ABORT_TIMEOUT = 1, ABORT_DONE = 2;
 // Bounded per-thread wait that also gives up when another role aborted. The
 // thread sleeps in the barrier (suspend hint) instead of spinning. (Out of line,
 // with scalar arguments only, so that callers keep their context in registers.)
+// (The bound lives in shared memory beside the abort word: MISC_WAIT_NS.)
 __device__ __noinline__ bool wait_b_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = *reinterpret_cast<const volatile uint64_t*>(
+      reinterpret_cast<volatile uint8_t*>(abort_flag) + MISC_WAIT_NS);
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > WAIT_NS) {
+    if (globaltimer_ns() - t0 > limit) {
       *abort_flag = ABORT_TIMEOUT;
       flag_error(DEVERR_TIMEOUT);
       return false;
@@ -1178,7 +1186,8 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
     fence_proxy_async_smem();
     named_bar_sync(BAR_PB, PB_THREADS);
     if (tid == 0) {
-      mbar_arrive(&x.bars[B_TB]);
+      // (a test may leave one arrive out: the state warps' wait for it then runs out)
+      if (c != *reinterpret_cast<const int*>(x.sm + OFF_MISC + MISC_SKIP_TB)) mbar_arrive(&x.bars[B_TB]);
       mbar_arrive(&x.bars[B_WFREE]);   // done with this chunk: the workspace is free
       push_kq(c + 2, false);
     }
@@ -1563,7 +1572,7 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   x.bars = reinterpret_cast<uint64_t*>(x.sm + OFF_BAR);
   x.abort_flag = reinterpret_cast<volatile int*>(x.sm + OFF_MISC);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x.sm + OFF_MISC + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(x.sm + OFF_MISC + MISC_TMEM);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = args.n_heads;
   const int slot = blockIdx.x / H;
@@ -1629,6 +1638,8 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   if (threadIdx.x == 0) {
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(&x.bars[i], 1);
     *x.abort_flag = 0;
+    *reinterpret_cast<uint64_t*>(x.sm + OFF_MISC + MISC_WAIT_NS) = args.wait_ns ? args.wait_ns : WAIT_NS;
+    *reinterpret_cast<int*>(x.sm + OFF_MISC + MISC_SKIP_TB) = args.debug_skip_tb;
     fence_mbar_init();
   }
   if (threadIdx.x == 0) {

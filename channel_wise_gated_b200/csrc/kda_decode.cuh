@@ -125,6 +125,14 @@ namespace kda {
 // together with the state's.
 constexpr int DEC_MAX_TOKENS = 16;
 
+// Shared memory of the multi-token step (dynamic: more than the 48 KB of static data).
+struct DecTokensSmem {
+  float k[DEC_MAX_TOKENS][D], q[DEC_MAX_TOKENS][D], a[DEC_MAX_TOKENS][D], v[DEC_MAX_TOKENS][D];
+  // the partial projections, double-buffered by token parity: one barrier per token
+  float4 u[2][DEC_THREADS / 32][32], y[2][DEC_THREADS / 32][32];
+  float beta[DEC_MAX_TOKENS], kq[DEC_MAX_TOKENS];
+};
+
 template <typename TQ, typename TG>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
 kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
@@ -136,10 +144,16 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  __shared__ float s_k[DEC_MAX_TOKENS][D], s_q[DEC_MAX_TOKENS][D];
-  __shared__ float s_a[DEC_MAX_TOKENS][D], s_v[DEC_MAX_TOKENS][D];
-  __shared__ float4 s_u[DEC_THREADS / 32][32], s_y[DEC_THREADS / 32][32];
-  __shared__ float s_beta[DEC_MAX_TOKENS];
+  extern __shared__ __align__(16) unsigned char dec_smem[];
+  DecTokensSmem& sm = *reinterpret_cast<DecTokensSmem*>(dec_smem);
+  auto& s_k = sm.k;
+  auto& s_q = sm.q;
+  auto& s_a = sm.a;
+  auto& s_v = sm.v;
+  auto& s_u = sm.u;
+  auto& s_y = sm.y;
+  auto& s_beta = sm.beta;
+  auto& s_kq = sm.kq;
 
   float4* S = reinterpret_cast<float4*>(state + (size_t)chain * D * D);
   const int row0 = warp * DEC_ROWS_PER_WARP;
@@ -162,40 +176,57 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
   TQ* od = o + ((size_t)seq * n_tokens * n_heads + h) * D + lane * 4;
   const size_t o_step = (size_t)n_heads * D;
   __syncthreads();
-
+  // k^T q of every token once (warp w takes tokens w, w + 8), formed exactly as the
+  // single step forms it; read after the first token's barrier
 #pragma unroll 1
-  for (int t = 0; t < n_tokens; ++t, od += o_step) {
-    // decay and the two partial projections over this warp's rows
-    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) {
-      const int r = row0 + i;
-      const float a = s_a[t][r], kr = s_k[t][r], qr = s_q[t][r];
-      s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
-      u.x = fmaf(kr, s[i].x, u.x); u.y = fmaf(kr, s[i].y, u.y);
-      u.z = fmaf(kr, s[i].z, u.z); u.w = fmaf(kr, s[i].w, u.w);
-      y.x = fmaf(qr, s[i].x, y.x); y.y = fmaf(qr, s[i].y, y.y);
-      y.z = fmaf(qr, s[i].z, y.z); y.w = fmaf(qr, s[i].w, y.w);
-    }
-    s_u[warp][lane] = u;
-    s_y[warp][lane] = y;
-
+  for (int t = warp; t < n_tokens; t += DEC_THREADS / 32) {
     float kq = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) kq = fmaf(s_k[t][lane * 4 + i], s_q[t][lane * 4 + i], kq);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    if (lane == 0) s_kq[t] = kq;
+  }
+
+#pragma unroll 1
+  for (int t = 0; t < n_tokens; ++t, od += o_step) {
+    const int buf = t & 1;
+    // decay and the two partial projections over this warp's rows (4 rows of the
+    // gates and keys per 16-byte read; rows in the single step's order)
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
+      const float4 a4 = *reinterpret_cast<const float4*>(&s_a[t][row0 + i4]);
+      const float4 k4 = *reinterpret_cast<const float4*>(&s_k[t][row0 + i4]);
+      const float4 q4 = *reinterpret_cast<const float4*>(&s_q[t][row0 + i4]);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w},
+                  qv[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i4 + e;
+        const float a = av[e], kr = kv[e], qr = qv[e];
+        s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+        u.x = fmaf(kr, s[i].x, u.x); u.y = fmaf(kr, s[i].y, u.y);
+        u.z = fmaf(kr, s[i].z, u.z); u.w = fmaf(kr, s[i].w, u.w);
+        y.x = fmaf(qr, s[i].x, y.x); y.y = fmaf(qr, s[i].y, y.y);
+        y.z = fmaf(qr, s[i].z, y.z); y.w = fmaf(qr, s[i].w, y.w);
+      }
+    }
+    s_u[buf][warp][lane] = u;
+    s_y[buf][warp][lane] = y;
+    // (this token's buffer was last read two tokens ago, before the previous barrier)
     __syncthreads();
 
     u = make_float4(0.f, 0.f, 0.f, 0.f);
     y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < DEC_THREADS / 32; ++w) {
-      const float4 a = s_u[w][lane], b = s_y[w][lane];
+      const float4 a = s_u[buf][w][lane], b = s_y[buf][w][lane];
       u.x += a.x; u.y += a.y; u.z += a.z; u.w += a.w;
       y.x += b.x; y.y += b.y; y.z += b.z; y.w += b.w;
     }
+    const float kq = s_kq[t];
     const float bt = s_beta[t];
     const float4 vv = reinterpret_cast<const float4*>(s_v[t])[lane];
     float4 dl;
@@ -209,12 +240,17 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
       od[3] = from_f32<TQ>(fmaf(kq, dl.w, y.w));
     }
 #pragma unroll
-    for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) {
-      const float kr = s_k[t][row0 + i];
-      s[i].x = fmaf(kr, dl.x, s[i].x); s[i].y = fmaf(kr, dl.y, s[i].y);
-      s[i].z = fmaf(kr, dl.z, s[i].z); s[i].w = fmaf(kr, dl.w, s[i].w);
+    for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
+      const float4 k4 = *reinterpret_cast<const float4*>(&s_k[t][row0 + i4]);
+      const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = i4 + e;
+        const float kr = kv[e];
+        s[i].x = fmaf(kr, dl.x, s[i].x); s[i].y = fmaf(kr, dl.y, s[i].y);
+        s[i].z = fmaf(kr, dl.z, s[i].z); s[i].w = fmaf(kr, dl.w, s[i].w);
+      }
     }
-    __syncthreads();   // s_u / s_y are rewritten by the next token
   }
 #pragma unroll
   for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) __stcs(&S[(row0 + i) * (D / 4) + lane], s[i]);
@@ -226,8 +262,12 @@ cudaError_t launch_decode_tokens(const TQ* q, const TQ* k, const TQ* v, const TG
                                  const TG* beta, float* state, TQ* o, int n_seqs, int n_tokens,
                                  int n_heads, cudaStream_t stream) {
   const unsigned chains = (unsigned)n_seqs * (unsigned)n_heads;
-  kda_decode_tokens_kernel<TQ, TG><<<chains, DEC_THREADS, 0, stream>>>(q, k, v, log_alpha, beta,
-                                                                       state, o, n_heads, n_tokens);
+  const size_t smem = sizeof(DecTokensSmem);
+  const cudaError_t e = cudaFuncSetAttribute(kda_decode_tokens_kernel<TQ, TG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kda_decode_tokens_kernel<TQ, TG><<<chains, DEC_THREADS, smem, stream>>>(
+      q, k, v, log_alpha, beta, state, o, n_heads, n_tokens);
   return cudaGetLastError();
 }
 

@@ -141,7 +141,8 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
  * KDA_ERR_CUDA if n_sms is 0 and the device cannot be queried). If seg_bounds is
  * not NULL and n >= 3, it receives n + 1 token offsets: segment j covers tokens
  * [seg_bounds[j], seg_bounds[j+1]), seg_bounds[0] = 0, seg_bounds[n] = t_total,
- * every inner offset a multiple of 64. At most KDA_MAX_SEGMENTS segments.
+ * every inner offset a multiple of 64, segments balanced to within one chunk, every
+ * segment at least 16 chunks. At most KDA_MAX_SEGMENTS segments.
  */
 #define KDA_MAX_SEGMENTS 64
 int kda_chunk_fwd_split_plan(int32_t n_heads, int64_t t_total, int32_t n_sms,
@@ -392,6 +393,27 @@ int kda_decode_tokens(const void* q, const void* k, const void* v, const void* l
  * from the others; synchronise the streams and read it once where that matters.
  */
 int kda_device_status(cudaStream_t stream);
+
+/*
+ * kda_testing_chunk_fwd_stall - TESTING ONLY: exercises the kernels' bounded waits.
+ * The pages have no counterpart; this entry point exists so that a test can make a wait
+ * run out without faulting or hanging the GPU.
+ *
+ * Runs kda_chunk_fwd's tensor-core kernel (one bf16 sequence, single pass) with every
+ * wait bounded by wait_us microseconds instead of 2 s, and with the producer of chunk
+ * skip_chunk's "T*beta ready" signal (a software mbarrier arrive; no copy or tensor-core
+ * completion is skipped) leaving that one arrive out. The consumer's wait then runs out:
+ * the kernel records KDA_ERR_TIMEOUT, every role leaves its loop, copies in flight are
+ * awaited and tensor memory is freed, and the call's outputs are undefined. Read the
+ * result with kda_device_status(). skip_chunk = -1 leaves nothing out.
+ * Arguments as kda_chunk_fwd for one sequence (cu_seqlens NULL, n_seqs 1, bf16).
+ * Returns KDA_OK (launched), KDA_ERR_SHAPE (t_total < 64 or wait_us = 0), or another
+ * negative kda_status.
+ */
+int kda_testing_chunk_fwd_stall(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, const float* h0,
+                                int64_t t_total, int32_t n_heads, void* o, float* hT,
+                                int32_t skip_chunk, uint32_t wait_us, cudaStream_t stream);
 
 /* kda_status_string - a static, human-readable name for a kda_status value. */
 const char* kda_status_string(int status);

@@ -568,10 +568,11 @@ def main():
     step_bytes = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + N * H * STATE_BYTES * (
         2 if inp["h0"] is not None else 1)
     # one prefill call = one launch of the chunk kernel, or, for one long sequence
-    # split in time, its state pass + the segment scan + its output pass
-    split = N == 1 and kda._native.load().kda_chunk_fwd_workspace_size(
-        1, T, H, kda._native.KDA_BF16, 0) > 0
-    launches_per_call = 3 if split else 1
+    # split in time, its zero-state pass + the segment scan (3 segments or more) + its
+    # correction pass
+    n_seg = len(kda.split_plan(H, T)) - 1 if N == 1 else 0
+    split = n_seg >= 2
+    launches_per_call = (3 if n_seg >= 3 else 2) if split else 1
 
     with ClockSampler(local) as clk:
         total_ms, per_launch = time_prefill(kda, inp, args.steps, args.warmup, ws, stream)
@@ -651,8 +652,9 @@ def main():
                                           " null if the kernel changed since"),
                          "peak_kind": peak_kind,
                          "kernel": "kda_chunk_tc_kernel",
-                         "unit_of_work": ("one prefill call (state pass + segment scan + "
-                                          "output pass)" if split else "one launch"),
+                         "unit_of_work": (f"one prefill call split in {n_seg} segments "
+                                          "(zero-state pass + segment scan + correction pass)"
+                                          if split else "one launch"),
                          "algorithmic_bytes_per_call": step_bytes,
                          "avg_call_ms": avg_launch_ms},
             "cpu_baseline": cpu,

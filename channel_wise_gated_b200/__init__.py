@@ -260,7 +260,7 @@ def split_plan(n_heads: int, t_total: int, n_sms: int = 0, workspace_bytes: Opti
     n = lib.kda_chunk_fwd_split_plan(int(n_heads), int(t_total), int(n_sms), ws, bounds)
     if n < 0:
         raise KdaError(n, "kda_chunk_fwd_split_plan")
-    return [int(bounds[i]) for i in range(n + 1)] if n >= 3 else []
+    return [int(bounds[i]) for i in range(n + 1)] if n >= 2 else []
 
 
 def decode_step(q, k, v, log_alpha, beta, state, o=None):

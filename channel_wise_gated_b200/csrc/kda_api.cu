@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -115,44 +116,45 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Time split of one long sequence (see the chunk kernel's plans). A split into n
-// segments runs H (2n - 3) CTAs in the state pass (n - 2 transition chains M_j,
-// n - 2 chains R_j and segment 0's output pass per head) and H (n - 1) in the
-// output pass, each over about n_chunks / n chunks, so a call costs about
-// 2 / n of the single pass when both passes fit one wave of SMs. The output pass
-// must fit one wave. The transition chains come first in the state pass and stop
-// as soon as their state is exactly zero; for segments of SPLIT_EARLY_CHUNKS
-// chunks or more the plan counts on that (the erase and the decay shrink every
-// direction of the state: with unit keys and beta near 0.5 the transition loses
-// about e^-0.2 per chunk even without decay, so it underflows to zero within a
-// few hundred chunks), and otherwise plans for the pass taking as many waves as
-// it has CTAs for. Every segment keeps at least MIN_SEG_CHUNKS chunks, and the
-// plan's scratch must fit the bytes available.
+// Every segment keeps at least MIN_SEG_CHUNKS chunks; at most MAX_SEGMENTS.
 constexpr int MIN_SEG_CHUNKS = 16;
 constexpr int MAX_SEGMENTS = 64;
 constexpr int64_t SPLIT_EARLY_CHUNKS = 512;
 
-size_t segment_workspace_bytes(int n_seg, int32_t n_heads) {
-  return n_seg >= 3 ? (size_t)kda::seg::slots(n_seg) * n_heads * kda::D * kda::D * sizeof(float) : 0;
+// Time split of one long sequence (the chunk kernel's PLAN_ZERO, the segment scan,
+// PLAN_CORR; see the kernel's plans). A split into n segments runs all n segments from
+// zero states side by side (H n CTAs, which must fit one wave), the n - 2 transition
+// chains per head on the SMs left over or after them, the scan (n - 2 products of
+// 128 x 128 matrices per head, about two chunk periods each), and n - 1
+// corrections per head. Transition chains and corrections both stop once their
+// state is exactly zero; for segments of SPLIT_EARLY_CHUNKS chunks or more the plan
+// counts on that within STOP_CHUNKS chunks, and otherwise on neither stopping. In
+// chunk periods a split costs one segment, plus the transition chains that do not
+// fit beside the segments, plus the scan, plus one correction; the single pass
+// costs the whole sequence. Every segment keeps at least MIN_SEG_CHUNKS chunks, and
+// the plan's scratch must fit the bytes available.
+constexpr int64_t STOP_CHUNKS = 64;
+constexpr double SCAN_STEP_CHUNKS = 2.0;
+
+size_t split_workspace_bytes(int n_seg, int32_t n_heads) {
+  return n_seg >= 2 ? (size_t)(2 * n_seg - 2) * n_heads * kda::D * kda::D * sizeof(float) : 0;
 }
 
-int split_segments(int32_t n_heads, int64_t n_chunks, int sms, size_t max_bytes) {
+int split_segments(int64_t n_chunks, int32_t n_heads, int sms, size_t max_bytes) {
+  if (sms <= 0 || n_heads <= 0) return 0;
   int best = 0;
-  double best_cost = 1.0;   // the single pass, in units of its own time
-  for (int n = 3; n <= MAX_SEGMENTS; ++n) {
+  double best_cost = (double)n_chunks * (double)((n_heads + sms - 1) / sms);
+  for (int n = 2; n <= MAX_SEGMENTS; ++n) {
     if (n_chunks < (int64_t)n * MIN_SEG_CHUNKS) break;
-    if ((int64_t)n_heads * (n - 1) > sms) break;
-    if (segment_workspace_bytes(n, n_heads) > max_bytes) break;
-    const double seg = 1.0 / n;
-    const int64_t ctas1 = (int64_t)n_heads * (2 * n - 3);
-    double pass1;
-    if (ctas1 <= sms)
-      pass1 = seg;
-    else if (n_chunks / n >= SPLIT_EARLY_CHUNKS)
-      pass1 = 1.05 * seg;
-    else
-      pass1 = seg * (double)((ctas1 + sms - 1) / sms);
-    const double cost = pass1 + seg;
+    if ((int64_t)n_heads * n > sms) break;
+    if (split_workspace_bytes(n, n_heads) > max_bytes) break;
+    const double len = (double)((n_chunks + n - 1) / n);
+    const double z = len >= (double)SPLIT_EARLY_CHUNKS ? std::min(len, (double)STOP_CHUNKS) : len;
+    const int64_t trans = (int64_t)n_heads * (n - 2), spare = sms - (int64_t)n_heads * n;
+    double extra = 0.0;
+    if (trans > 0 && (spare == 0 || (double)((trans + spare - 1) / spare) * z > len))
+      extra = z * (double)((trans + sms - 1) / sms);
+    const double cost = len + extra + SCAN_STEP_CHUNKS * (n - 2) + z;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = n;
@@ -252,33 +254,48 @@ int launch_chunk_tc(const void* q, const void* k, const void* v, const float* lo
     if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
     a.seq_order = seq_order;
   }
-  if (n_seg < 3 || seg_states == nullptr) {
+  if (n_seg < 2 || seg_states == nullptr) {
     const int64_t grid = (int64_t)n_seqs * n_heads;   // one CTA per (sequence, head)
     kda_chunk_tc_kernel<false, MODE><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(mk, mq, mv, mla, mo, a);
     return launch_status();
   }
-  // time split: segment states (with segment 0's output), the scan over segments,
-  // then the outputs of segments 1 .. n-1
+  // time split: every segment from a zero state (segment 0 from h0) with its output
+  // and the transition chains, the scan over segments, then the corrections of
+  // segments 1 .. n-1 (and for the fused variant the norm and gate of their outputs)
   const int64_t n_chunks = (t_total + kda::CHUNK - 1) / kda::CHUNK;
   a.n_seg = n_seg;
   a.seg_base = (int)(n_chunks / n_seg);
   a.seg_rem = (int)(n_chunks % n_seg);
   a.seg_states = seg_states;
-  a.plan = PLAN_STATES;
-  kda_chunk_tc_kernel<true, MODE><<<(unsigned)(n_heads * (2 * n_seg - 3)), THREADS, SMEM_BYTES, stream>>>(
+  a.plan = PLAN_ZERO;
+  kda_chunk_tc_kernel<true, MODE><<<(unsigned)(n_heads * (2 * n_seg - 2)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
   if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
-  if (cudaFuncSetAttribute(kda::seg::kda_segment_scan_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kda::seg::SCAN_SMEM) != cudaSuccess)
-    return KDA_ERR_CUDA;
-  kda::seg::kda_segment_scan_kernel<<<(unsigned)n_heads, kda::seg::SCAN_THREADS, kda::seg::SCAN_SMEM,
-                                       stream>>>(seg_states, n_heads, n_seg);
-  if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
-  a.plan = PLAN_OUTPUTS;
-  kda_chunk_tc_kernel<false, MODE><<<(unsigned)(n_heads * (n_seg - 1)), THREADS, SMEM_BYTES, stream>>>(
+  if (n_seg >= 3) {
+    if (cudaFuncSetAttribute(kda::seg::kda_segment_scan_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kda::seg::SCAN_SMEM) != cudaSuccess)
+      return KDA_ERR_CUDA;
+    kda::seg::kda_segment_scan_kernel<<<(unsigned)n_heads, kda::seg::SCAN_THREADS, kda::seg::SCAN_SMEM,
+                                         stream>>>(seg_states, n_heads, n_seg);
+    if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
+  }
+  a.plan = PLAN_CORR;
+  kda_chunk_tc_kernel<true, MODE><<<(unsigned)(n_heads * (n_seg - 1)), THREADS, SMEM_BYTES, stream>>>(
       mk, mq, mv, mla, mo, a);
-  return launch_status();
+  if (launch_status() != KDA_OK) return KDA_ERR_CUDA;
+  if constexpr (MODE == MODE_FUSED) {
+    const int64_t t1 = kda::seg::seg_first_chunk(1, a.seg_base, a.seg_rem) * kda::CHUNK;
+    const int64_t rows = (t_total - t1) * n_heads;
+    const int64_t want = (rows + NG_ROWS - 1) / NG_ROWS;
+    const int sms = device_sms();
+    const int64_t cap = (int64_t)(sms > 0 ? sms : 148) * 16;
+    kda_norm_gate_kernel<<<(unsigned)(want < cap ? want : cap), NG_THREADS, 0, stream>>>(
+        static_cast<__nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(fu->gate_pre), fu->norm_w,
+        t1 * n_heads, rows);
+    return launch_status();
+  }
+  return KDA_OK;
 }
 
 // Whether a call takes the tensor-core path and, if so, how many segments it splits into.
@@ -295,7 +312,7 @@ int plan_segments(const int32_t* cu_seqlens, int32_t n_seqs, int64_t t_total, in
                   kda_dtype qkv_dtype, size_t max_bytes) {
   if (!use_tc(cu_seqlens, n_seqs, t_total, n_heads, qkv_dtype) || cu_seqlens != nullptr || n_seqs != 1)
     return 0;
-  return split_segments(n_heads, (t_total + kda::CHUNK - 1) / kda::CHUNK, device_sms(), max_bytes);
+  return split_segments((t_total + kda::CHUNK - 1) / kda::CHUNK, n_heads, device_sms(), max_bytes);
 }
 
 template <typename TQ, typename TG>
@@ -423,9 +440,9 @@ size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_h
                                     kda_dtype qkv_dtype, int has_cu_seqlens) {
   if (n_heads <= 0 || n_seqs <= 0 || t_total < 0) return 0;
   static const int32_t dummy = 0;
-  const int n_seg = plan_segments(has_cu_seqlens ? &dummy : nullptr, n_seqs, t_total, n_heads,
-                                  qkv_dtype, SIZE_MAX);
-  if (n_seg >= 3) return segment_workspace_bytes(n_seg, n_heads);
+  const int32_t* cu = has_cu_seqlens ? &dummy : nullptr;
+  const int n_seg = plan_segments(cu, n_seqs, t_total, n_heads, qkv_dtype, SIZE_MAX);
+  if (n_seg >= 2) return split_workspace_bytes(n_seg, n_heads);
   if (has_cu_seqlens && n_seqs > 1 &&
       use_tc(&dummy, n_seqs, t_total, n_heads, qkv_dtype))
     return order_workspace_bytes(n_seqs, n_heads);
@@ -439,8 +456,8 @@ int kda_chunk_fwd_split_plan(int32_t n_heads, int64_t t_total, int32_t n_sms,
   if (n_sms <= 0) return KDA_ERR_CUDA;
   if (!use_tc(nullptr, 1, t_total, n_heads, KDA_BF16)) return 0;
   const int64_t n_chunks = (t_total + kda::CHUNK - 1) / kda::CHUNK;
-  const int n_seg = split_segments(n_heads, n_chunks, n_sms, workspace_bytes);
-  if (n_seg >= 3 && seg_bounds != nullptr) {
+  const int n_seg = split_segments(n_chunks, n_heads, n_sms, workspace_bytes);
+  if (n_seg >= 2 && seg_bounds != nullptr) {
     const int base = (int)(n_chunks / n_seg), rem = (int)(n_chunks % n_seg);
     for (int j = 0; j < n_seg; ++j) seg_bounds[j] = kda::seg::seg_first_chunk(j, base, rem) * kda::CHUNK;
     seg_bounds[n_seg] = t_total;

@@ -161,28 +161,38 @@ enum : int {
 static_assert(NUM_BARS <= NBARS, "barrier slots");
 
 // Work plans. PLAN_SEQ: one CTA per (sequence of cu_seqlens, head). The time split
-// of one long sequence cuts it into n_seg segments of whole chunks, balanced to
-// within one chunk (segment j starts at chunk j*seg_base + min(j, seg_rem); the
-// last one ends at t_total), and runs as PLAN_STATES, the segment scan, then
-// PLAN_OUTPUTS. Slots of seg_states [2 n_seg - 3][H][128][128]: slot 0 the state
-// entering segment 1; slot j (1 .. n_seg-2) R_j, the final state of segment j from
-// a zero start, which the scan overwrites with the state entering segment j+1;
-// slot n_seg-2+j the transition M_j of segment j (S_end = M_j S_start + R_j).
-//   PLAN_STATES (grid H x (2 n_seg - 3)), in block order:
-//     M_1 .. M_{n-2}   segment j from the identity with v = 0: its final state is
-//                      M_j. These come first and end early: once the state is
-//                      exactly zero it stays zero, so the CTA stops there.
-//     R_1 .. R_{n-2}   segment j from a zero state
-//     O_0              segment 0 from the caller's h0, writing its output; its
-//                      final state goes to slot 0
-//   The M and R CTAs write no output and run the lean form of every role (a
-//   CTA-uniform flag, not a second kernel: all CTAs run one body of code, so that
-//   SMs sharing instruction caches fetch the same code): no q loads, no Rq tile, no
-//   P readout, the state product only for Delta (N=64), no P Delta product; with
-//   v = 0 also no U product.
-//   PLAN_OUTPUTS (grid H x (n_seg - 1)): segment j = 1 .. n_seg-1 from slot j-1,
-//     writing o, and the caller's hT for the last segment.
-enum : int { PLAN_SEQ = 0, PLAN_STATES = 1, PLAN_OUTPUTS = 2 };
+// of one long sequence cuts it into n_seg >= 2 segments of whole chunks, balanced to
+// within one chunk (segment j starts at chunk j*seg_base + min(j, seg_rem); the last
+// one ends at t_total). Every step of the recurrence is affine in the state, so a
+// segment maps its entering state S to M S + R (M the product of its transitions, R
+// its final state from a zero start), and its output is its output from a zero
+// start plus the output of the same segment run from S with v = 0 (the correction).
+// Slots of seg_states [2 n_seg - 2][H][128][128]. The split runs
+//   PLAN_ZERO (grid H x (2 n_seg - 2)), in block order:
+//     Z_0 .. Z_{n-1}   every segment from a zero state (segment 0 from the caller's
+//                      h0), storing its output; final states: segment 0's to slot
+//                      0, R_j to slot j (j = 1 .. n-2), R_{n-1} to slot 2 n_seg - 3
+//     M_1 .. M_{n-2}   segment j from the identity with v = 0, output discarded: its
+//                      final state is M_j (slot n_seg - 2 + j). Once the state is
+//                      exactly zero it stays zero, so the CTA stops there. These
+//                      take the SMs the Z CTAs leave free, or follow them.
+//   the segment scan (slot j <- S_{j+1} = M_j S_j + R_j), then
+//   PLAN_CORR (grid H x (n_seg - 1)): segment j = 1 .. n_seg-1 from slot j-1 with
+//     v = 0, adding its output onto o and stopping once its state is exactly zero
+//     (every later correction is zero); for the last segment the caller's hT =
+//     R_{n-1} + the chain's final state (zero after a stop).
+// With typical decay the corrections die out within some tens of chunks, so a call
+// costs about one pass over 1/n_seg of the sequence; without decay or erase they run
+// to the ends of their segments (two such passes). The fused variant's output is not
+// linear in o (its RMSNorm): in the split only segment 0's CTAs apply the norm and
+// the gate, the other Z CTAs and the corrections work on the raw output, and a last
+// pass (kda_norm_gate_kernel) normalises and gates segments 1 .. n-1.
+// The kernel's SPLIT instance serves PLAN_ZERO and PLAN_CORR and reads the per-CTA
+// flags below; the PLAN_SEQ instance has them all off at compile time.
+enum : int { PLAN_SEQ = 0, PLAN_ZERO = 1, PLAN_CORR = 2 };
+// What a CTA does with its output: store it, discard it (a transition chain), or
+// add it onto o (a correction)
+enum : int { OUT_STORE = 0, OUT_NONE = 1, OUT_ADD = 2 };
 
 struct Args {
   const float* log_alpha;
@@ -197,7 +207,7 @@ struct Args {
   int plan;
   int n_seg;
   int seg_base, seg_rem;   // chunks per segment: seg_base, plus one for the first seg_rem
-  float* seg_states;   // [2 n_seg - 3][H][128][128]
+  float* seg_states;   // [2 n_seg - 2][H][128][128]
   const int32_t* seq_order;   // PLAN_SEQ: sequences longest first (or null: index order)
   // MODE_FUSED: log_alpha and beta are unused; these take their place
   const __nv_bfloat16* decay_pre;   // [T, H, 128], log alpha = logsigmoid(decay_pre)
@@ -220,17 +230,14 @@ struct Ctx {
   size_t rs;          // elements between consecutive tokens of q/k/v/o/log_alpha
   const float* h0;    // this CTA's entering state [channel][value], or null (zeros)
   float* hT;          // where its final state goes, or null
+  const float* hT_base;   // if not null: hT = hT_base + the final state
   bool h0_identity;   // entering state = I (transition of a segment)
   bool v_zero;        // v taken as zero (no loads)
-  bool write_o;       // store the output
-  bool stop_on_zero;  // a transition chain: stop once the state is exactly zero
-  bool lean;          // no output: the lean form of every role
+  int out_mode;       // OUT_STORE, OUT_NONE or OUT_ADD
+  bool stop_on_zero;  // stop once the state is exactly zero (v = 0 chains)
+  bool gated;         // MODE_FUSED: the output is final (RMSNorm and gate applied)
 };
 
-// Whether a CTA runs the lean form of the roles. RT = false compiles the full form
-// only (every CTA writes output); RT = true reads the CTA's flag.
-template <bool RT>
-__device__ __forceinline__ bool lean_of(const Ctx& x) { return RT && x.lean; }
 
 // Values of the shared abort word: a role that gives up a wait raises ABORT_TIMEOUT
 // (and flags the device error); the state warps of a transition chain raise
@@ -405,7 +412,6 @@ __device__ __forceinline__ uint64_t kdesc128(uint32_t addr) {
 // ============================================================================
 // TMA and MMA issue (each by the first thread of the role that consumes the result)
 // ============================================================================
-template <bool RT>
 __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* map_k,
                                          const CUtensorMap* map_q, int c) {
   const int xk = x.h * D;
@@ -413,18 +419,18 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* map_k,
   uint8_t* st = x.sm + OFF_KQ + (c % 3) * KQ_BYTES;
   const uint32_t koff = (c & 1) ? 8192u : 0u, qoff = 8192u - koff;
   uint64_t* full = &x.bars[B_FULL + c % 3];
-  mbar_arrive_expect_tx(full, (lean_of<RT>(x) ? 2 : 4) * 8192);
+  mbar_arrive_expect_tx(full, 4 * 8192);
   tma_load_2d(st + koff, map_k, xk, y, full);
   tma_load_2d(st + 16384 + koff, map_k, xk + 64, y, full);
-  if (lean_of<RT>(x)) return;   // no output: q is not needed
   tma_load_2d(st + qoff, map_q, xk, y, full);
   tma_load_2d(st + 16384 + qoff, map_q, xk + 64, y, full);
 }
+template <bool SPLIT>
 __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* map_v, int c) {
   const int xk = x.h * D;
   const int y = (int)(x.bos + (int64_t)c * CHUNK);
   uint64_t* full = &x.bars[B_VFULL];
-  if (x.v_zero) {   // the v tile stays zero: complete the phase without a copy
+  if (SPLIT && x.v_zero) {   // the v tile stays zero: complete the phase without a copy
     mbar_arrive(full);
     return;
   }
@@ -445,26 +451,15 @@ __device__ void drain(const Ctx& x, int bar) {
 }
 
 // [O | Delta]^T (or [Delta | O]^T) += S''^T [stage tile]^T   (M=128, N=128, K=128);
-// the state operand comes from TMEM. Without output (lean) only Delta^T += S''^T (-W')^T
-// (N=64); with v = 0 there is no U to accumulate onto.
-template <bool RT>
+// the state operand comes from TMEM
 __device__ __forceinline__ void issue_crit(const Ctx& x, int c) {
   tc_fence_after();
   const uint32_t kq = smem_u32(x.sm) + OFF_KQ + (c % 3) * KQ_BYTES;
-  if (lean_of<RT>(x)) {
-    const uint32_t kh = kq + ((c & 1) ? 8192u : 0u);
+  const uint32_t d = x.tmem + ((c & 1) ? TM_OA : TM_D);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      umma_bf16_tmem_a(x.tmem + TM_D, x.tmem + TM_SB + kk * 8,
-                       kdesc128(kh + (kk >> 2) * 16384 + (kk & 3) * 32), IDESC_DELTA,
-                       (kk == 0 && x.v_zero) ? 0u : 1u);
-  } else {
-    const uint32_t d = x.tmem + ((c & 1) ? TM_OA : TM_D);
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      umma_bf16_tmem_a(d, x.tmem + TM_SB + kk * 8, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
-                       IDESC_CRIT, 1u);
-  }
+  for (int kk = 0; kk < 8; ++kk)
+    umma_bf16_tmem_a(d, x.tmem + TM_SB + kk * 8, kdesc128(kq + (kk >> 2) * 16384 + (kk & 3) * 32),
+                     IDESC_CRIT, 1u);
   umma_commit(&x.bars[B_CRIT]);
   umma_commit(&x.bars[B_KQFREE + c % 3]);
 }
@@ -473,9 +468,8 @@ __device__ __forceinline__ void issue_crit(const Ctx& x, int c) {
 // 32-63 into its last 16, each warp inside the columns it has just read
 __device__ __forceinline__ uint32_t dpair_col(int kk) { return TM_D + (kk < 2 ? 8 * kk : 48 + 8 * (kk - 2)); }
 
-// S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T (not without output);
-// Delta^T is the A operand, read from TMEM
-template <bool RT>
+// S^T += Delta^T Ck (the state update), then O^T += Delta^T P^T; Delta^T is the A
+// operand, read from TMEM
 __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   tc_fence_after();
   const uint32_t sbase = smem_u32(x.sm);
@@ -486,10 +480,6 @@ __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
     umma_bf16_tmem_a(x.tmem + TM_S, x.tmem + dpair_col(kk),
                      make_sdesc(ck + kk * 2048, 8192, 1024, SWZ_128B), IDESC_Z, 1u);
   umma_commit(&x.bars[B_ZDONE]);
-  if (lean_of<RT>(x)) {
-    umma_commit(&x.bars[B_CKFREE + (c & 1)]);
-    return;
-  }
   // (M=128, N=64, K=64)
   const uint32_t o = x.tmem + ((c & 1) ? TM_OA : TM_OB);
 #pragma unroll
@@ -498,13 +488,9 @@ __device__ __forceinline__ void issue_update(const Ctx& x, int c) {
   umma_commit(&x.bars[B_PD]);
   umma_commit(&x.bars[B_CKFREE + (c & 1)]);
 }
-// U^T = V^T (T beta)^T   (M=128 value columns, N=64, K=64); v read as MN-major A
-template <bool RT>
+// U^T = V^T (T beta)^T   (M=128 value columns, N=64, K=64); v read as MN-major A (a
+// zero tile for a v = 0 chain: U = 0, which the [O | Delta] product accumulates onto)
 __device__ __forceinline__ void issue_u(const Ctx& x) {
-  if (lean_of<RT>(x) && x.v_zero) {   // U = 0: nothing to compute (the Delta product starts from zero)
-    umma_commit(&x.bars[B_UDONE]);
-    return;
-  }
   tc_fence_after();
   const uint32_t sbase = smem_u32(x.sm);
   const uint32_t tb = sbase + OFF_TB, vv = sbase + OFF_V;
@@ -703,7 +689,7 @@ __device__ __noinline__ bool prep_a_exact(const Ctx x, const float* log_alpha,
   return true;
 }
 
-template <bool RT, int MODE>
+template <bool SPLIT, int MODE>
 __device__ void prep_a_role(const Ctx& x, const Args& p) {
   constexpr bool SG = MODE == MODE_GDN, FU = MODE == MODE_FUSED;
   const int tid = threadIdx.x;
@@ -806,18 +792,15 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
     bool ok = wait_b(x, B_FULL + s3, (c / 3) & 1);
     if (named_bar_or(BAR_PA, PA_THREADS, !ok)) break;
     if (FU) {
-      // L2-normalise this warp's 8 rows of k (and q) in place: the 32 lanes hold the
+      // L2-normalise this warp's 8 rows of k and q in place: the 32 lanes hold the
       // 128 channels of a row, 4 each. All 16 row sums first, then their butterflies
       // side by side (independent shuffle chains), then the rescaled rows written back;
       // everything downstream reads the unit rows.
-      const bool do_q = !lean_of<RT>(x);
       float ss[2][8];
 #pragma unroll
       for (int half = 0; half < 2; ++half)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          ss[half][j] = 0.f;
-          if (half == 1 && !do_q) continue;
           const uint2 v = *reinterpret_cast<const uint2*>(kq + (half ? qoff : koff) + kb * 16384 +
                                                           swz128((8 * w + j) * 128 + cbyte));
           const float f0 = bf_lo(v.x), f1 = bf_hi(v.x), f2 = bf_lo(v.y), f3 = bf_hi(v.y);
@@ -833,7 +816,6 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
       for (int half = 0; half < 2; ++half)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          if (half == 1 && !do_q) continue;
           uint2* pp = reinterpret_cast<uint2*>(kq + (half ? qoff : koff) + kb * 16384 +
                                                swz128((8 * w + j) * 128 + cbyte));
           const uint2 v = *pp;
@@ -864,7 +846,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
         uint2* kp = reinterpret_cast<uint2*>(kq + koff + kb * 16384 + swz128(r * 128 + cbyte));
         uint2* qp = reinterpret_cast<uint2*>(kq + qoff + kb * 16384 + swz128(r * 128 + cbyte));
         const uint2 kr = valid ? *kp : make_uint2(0u, 0u);
-        const uint2 qv = (valid && !lean_of<RT>(x)) ? *qp : make_uint2(0u, 0u);
+        const uint2 qv = valid ? *qp : make_uint2(0u, 0u);
         float e[4], f[4];
         if (SG) {   // one factor per row
           e[0] = ex2f(g2[j][0] - gc[0]);
@@ -883,8 +865,7 @@ __device__ void prep_a_role(const Ctx& x, const Args& p) {
         }
         const uint32_t e01 = pack_bf16(e[0], e[1]), e23 = pack_bf16(e[2], e[3]);
         *kp = make_uint2(mul_bf16x2(kr.x, e01), mul_bf16x2(kr.y, e23));
-        if (!lean_of<RT>(x))   // Rq only where there is an output
-          *qp = make_uint2(mul_bf16x2(qv.x, e01), mul_bf16x2(qv.y, e23));
+        *qp = make_uint2(mul_bf16x2(qv.x, e01), mul_bf16x2(qv.y, e23));
         if (ok)
           *reinterpret_cast<uint2*>(ck + kb * 8192 + swz128(r * 128 + cbyte)) =
               make_uint2(mul_bf16x2(kr.x, pack_bf16(f[0], f[1])),
@@ -969,7 +950,7 @@ __device__ __forceinline__ void blk_store_tb(uint8_t* tt, int a, int b, const fl
   }
 }
 
-template <bool RT, int MODE>
+template <bool SPLIT, int MODE>
 __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtensorMap* map_q,
                             const CUtensorMap* map_la) {
   constexpr bool SG = MODE == MODE_GDN;
@@ -995,7 +976,7 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
         const uint32_t par = ((cn - 3) / 3) & 1;
         if (block ? !wait_b(x, B_KQFREE + cn % 3, par) : !mbar_test_wait(fb, par)) return;
       }
-      issue_kq<RT>(x, map_k, map_q, cn);
+      issue_kq(x, map_k, map_q, cn);
       // (a scalar gate is prefetched by prep A itself)
       if (!SG && cn + 3 < x.n_chunks)
         tma_prefetch_2d(map_la, xk, (int)(x.bos + (int64_t)(cn + 3) * CHUNK));
@@ -1046,7 +1027,7 @@ __device__ void prep_b_role(const Ctx& x, const CUtensorMap* map_k, const CUtens
             o4.w = (col0 + m + 3 < r) ? br * v[m + 3] : 0.f;
             *reinterpret_cast<float4*>(&aw[r * AW + col0 + m]) = o4;
           }
-        } else if (!lean_of<RT>(x)) {   // (P only where there is an output)
+        } else {
           uint8_t* pt = ck + 16384;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -1221,14 +1202,19 @@ __device__ __noinline__ void st_load_state(uint32_t lane_addr, const float* h0, 
   }
   tmem_st_wait();
 }
-// the final state out of the fp32 master
-__device__ __noinline__ void st_store_state(uint32_t lane_addr, float* hT, int j, int cb) {
+// the final state out of the fp32 master (plus base, if not null)
+__device__ __noinline__ void st_store_state(uint32_t lane_addr, float* hT, const float* base, int j,
+                                            int cb) {
 #pragma unroll 1
   for (int part = 0; part < 2; ++part) {
     const int cb0 = cb + 32 * part;
     float v[32];
     tmem_ld32(lane_addr + cb0, v);
     tmem_ld_wait();
+    if (base) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] += __ldg(base + (size_t)(cb0 + i) * D + j);
+    }
 #pragma unroll
     for (int i = 0; i < 32; ++i) hT[(size_t)(cb0 + i) * D + j] = v[i];
   }
@@ -1242,6 +1228,28 @@ __device__ __noinline__ void st_store_ragged(uint32_t lane_addr, __nv_bfloat16* 
 #pragma unroll
   for (int i = 0; i < 32; ++i)
     if (r0 + i < L) ocol[(size_t)(r0 + i) * rs] = __float2bfloat16_rn(v[i]);
+}
+
+// output rows r0..r0+31 (the valid rows < L only) added onto o: orow = o at the chunk's
+// first row and the head's first column; j = this thread's column. Adjacent columns
+// pair up through one shuffle (the even lane takes rows r0..r0+15, the odd lane
+// rows r0+16..) for bf16x2 atomic adds.
+__device__ __noinline__ void st_add_rows(uint32_t lane_addr, __nv_bfloat16* orow, size_t rs, int j,
+                                         int r0, int L) {
+  float v[32];
+  tmem_ld32(lane_addr, v);
+  tmem_ld_wait();
+  const bool odd = (j & 1) != 0;
+  __nv_bfloat16* col = orow + (j & ~1);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float mine = odd ? v[16 + i] : v[i];
+    const float other = __shfl_xor_sync(0xffffffffu, odd ? v[i] : v[16 + i], 1);
+    const int r = r0 + (odd ? 16 + i : i);
+    if (r < L)
+      atomicAdd(reinterpret_cast<__nv_bfloat162*>(col + (size_t)r * rs),
+                odd ? __floats2bfloat162_rn(other, mine) : __floats2bfloat162_rn(mine, other));
+  }
 }
 
 // ============================================================================
@@ -1262,7 +1270,7 @@ __device__ __forceinline__ uint4 gate_row8(uint4 o8, uint4 g8, const float* w8, 
   return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
-template <bool RT, int MODE>
+template <bool SPLIT, int MODE>
 __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v,
                            const CUtensorMap* map_o) {
   constexpr bool FU = MODE == MODE_FUSED;
@@ -1280,13 +1288,11 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   float* rowsq = reinterpret_cast<float*>(x.sm + OFF_ROWSQ);
   float* normw = reinterpret_cast<float*>(x.sm + OFF_NORMW);
   if (FU && tid < D) normw[tid] = __ldg(p.norm_w + tid);
-  st_load_state(x.tmem + TM_S + lb, x.h0, x.h0_identity, j, 64 * hh);
-  if (!lean_of<RT>(x)) {
-    tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
-    tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
-    tmem_st_wait();
-  }
-  if (x.v_zero) {   // a zero v tile for every chunk (U = 0)
+  st_load_state(x.tmem + TM_S + lb, x.h0, SPLIT && x.h0_identity, j, 64 * hh);
+  tmem_st32_zero(x.tmem + TM_OA + lb + 32 * hh);
+  tmem_st32_zero(x.tmem + TM_OB + lb + 32 * hh);
+  tmem_st_wait();
+  if (SPLIT && x.v_zero) {   // a zero v tile for every chunk (U = 0)
     for (int i = tid; i < 1024; i += ST_THREADS)
       *reinterpret_cast<uint4*>(x.sm + OFF_V + i * 16) = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
@@ -1305,7 +1311,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       float v[32];
       tmem_ld32(x.tmem + TM_S + lb + cb0, v);
       tmem_ld_wait();
-      if (RT && x.stop_on_zero) {
+      if (SPLIT && x.stop_on_zero) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) nz |= __float_as_uint(v[i]) & 0x7FFFFFFFu;
       }
@@ -1360,7 +1366,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       return true;   // not ready yet: issued later, before the chunk's [O | Delta] product
     }
     v_landed = cu + 1;
-    issue_u<RT>(x);
+    issue_u(x);
     u_issued = cu + 1;
     return true;
   };
@@ -1377,10 +1383,14 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
     return true;
   };
 
+  // output: the fused epilogue (RMSNorm and gate) where the output is final, else the
+  // plain one in the CTA's mode
+  const bool fu_out = FU && (!SPLIT || x.gated);
+  const int omode = SPLIT ? x.out_mode : OUT_STORE;
   bool alive = true;
-  bool stopped = false;   // a transition chain that stopped early (state exactly zero)
+  bool stopped = false;   // a v = 0 chain that stopped early (state exactly zero)
   if (issuer && n > 0) {
-    issue_v(x, map_v, 0);
+    issue_v<SPLIT>(x, map_v, 0);
     v_issued = 1;
   }
   // One pass of the loop per chunk c, plus one to finish the last output. Each step
@@ -1390,6 +1400,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   //   (b) the output of chunk c-1, off the sequential path;
   //   (c) Delta of chunk c back into TMEM as bf16 pairs, then the state update.
   for (int c = 0; c <= n; ++c) {
+    bool stop_now = false;
     if (c < n) {
       alive = alive && (c == 0 || wait_b(x, B_ZDONE, (c - 1) & 1)) &&
               wait_b(x, B_TILES + (c & 1), (c >> 1) & 1);
@@ -1402,25 +1413,25 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       alive = alive && w_readout(c);
       // (the output tile's last store must have read it before (b) stages the next)
       if (issuer && c > 1) bulk_wait_read_all();
-      if (RT && x.stop_on_zero && c > 0) {
-        // A transition chain whose state is exactly zero after chunk c-1 stays zero
-        // (v = 0, so every later Delta and update is zero too): its final state is
-        // known, and the CTA stops here. The other roles see ABORT_DONE at their
-        // next wait and leave; the update of chunk c-1 has landed.
+      if (SPLIT && x.stop_on_zero && c > 0) {
+        // A v = 0 chain whose state is exactly zero after chunk c-1 stays zero (every
+        // later Delta, update and output is zero too): its final state is known, and
+        // the CTA stops once the output of chunk c-1 is out. The other roles then
+        // see ABORT_DONE at their next wait and leave; the update of chunk c-1 has
+        // landed.
         if (!named_bar_or(BAR_ST, ST_THREADS, nonzero || !alive)) {
-          if (tid == 0) *x.abort_flag = ABORT_DONE;
           stopped = true;
-          break;
+          stop_now = true;
         }
       } else {
         named_bar_sync(BAR_ST, ST_THREADS);
       }
-      if (issuer && alive) {
+      if (issuer && alive && !stop_now) {
         if (u_issued < c + 1) alive = issue_u_of(c, true);
-        if (alive) issue_crit<RT>(x, c);
+        if (alive) issue_crit(x, c);
       }
     }
-    if (FU && c > 0 && !lean_of<RT>(x)) {
+    if (fu_out && c > 0) {
       // ---- fused output of chunk c-1: RMSNorm over each row's 128 values, times the
       //      weight and the sigmoid gate. (i) every warp stages its 32 x 32 block as
       //      bf16 and leaves the fp32 row sums of squares; (ii) after the group's
@@ -1476,29 +1487,35 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         bulk_commit_group();
       }
     }
-    if (!FU && c > 0 && !lean_of<RT>(x)) {
+    if (!fu_out && c > 0) {
       const int co = c - 1;
       const int64_t t0 = x.bos + (int64_t)co * CHUNK;
       const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
+      // (a full chunk to be stored goes through the output tile and one TMA store)
+      const bool tile_out = L == CHUNK && omode == OUT_STORE;
       alive = alive && wait_b(x, B_PD, co & 1);
       if (alive) {
         tc_fence_after();
         const uint32_t ro = (co & 1) ? TM_OA : TM_OB;
-        if (L == CHUNK) {
+        if (tile_out) {
           // full chunk: into the output tile (its previous store has read it), then one
           // TMA store of [64 rows][128 columns]
           tmem_block_to_tile_t(x.tmem + ro + lb + 32 * hh, 32 * qd, 32 * hh, dt, 8192u, lane);
           fence_proxy_async_smem();
-        } else {
+        } else if (omode == OUT_STORE) {
           // ragged last chunk of a sequence: direct stores of the valid rows only
           st_store_ragged(x.tmem + ro + lb + 32 * hh, p.o + (size_t)t0 * x.rs + x.h * D + j, x.rs,
                           32 * hh, L);
+        } else if (omode == OUT_ADD) {
+          // a correction: added onto the stored output, valid rows only
+          st_add_rows(x.tmem + ro + lb + 32 * hh, p.o + (size_t)t0 * x.rs + x.h * D, x.rs, j,
+                      32 * hh, L);
         }
         tmem_st32_zero(x.tmem + ro + lb + 32 * hh);
         tmem_st_wait();
         tc_fence_before();
       }
-      if (L == CHUNK) {
+      if (tile_out) {
         // the warps that do not issue only report their part staged and go on; the
         // issuing warp waits for all parts and sends the tile
         if (sw != 0) {
@@ -1512,6 +1529,10 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
           }
         }
       }
+    }
+    if (stop_now) {
+      if (tid == 0) *x.abort_flag = ABORT_DONE;
+      break;
     }
     if (c < n) {
       // ---- Delta^T fp32 (TMEM, chunk rows 32hh..32hh+31 of lane j) -> bf16 pairs in the
@@ -1529,13 +1550,13 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         tmem_st_wait();
         tc_fence_before();
         if (issuer && c + 1 < n) {   // U(c) is done: v of the next chunk may land
-          issue_v(x, map_v, c + 1);
+          issue_v<SPLIT>(x, map_v, c + 1);
           v_issued = c + 2;
         }
       }
       named_bar_sync(BAR_ST, ST_THREADS);
       if (issuer && alive) {
-        issue_update<RT>(x, c);
+        issue_update(x, c);
         if (c + 1 < n) {
           alive = issue_w_of(c + 1, false);
           if (alive && w_issued == c + 2) alive = issue_u_of(c + 1, false);
@@ -1547,7 +1568,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
   if (n > 0 && !stopped) alive = alive && wait_b(x, B_ZDONE, (n - 1) & 1);
   tc_fence_after();
   if (x.hT && alive && *x.abort_flag != ABORT_TIMEOUT)
-    st_store_state(x.tmem + TM_S + lb, x.hT, j, 64 * hh);
+    st_store_state(x.tmem + TM_S + lb, x.hT, SPLIT ? x.hT_base : nullptr, j, 64 * hh);
   if (issuer) {
     bulk_wait_all();
     drain(x, B_FIN_C);
@@ -1562,7 +1583,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
 // activations in prep A and the output's RMSNorm and gate in the state warps'
 // epilogue. The chunk algebra in between is the same for all three.
 // ============================================================================
-template <bool RT, int MODE>
+template <bool SPLIT, int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
 kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_la,
@@ -1579,10 +1600,11 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.h = blockIdx.x % H;
   x.rs = (size_t)H * D;
   x.h0_identity = false;
+  x.hT_base = nullptr;
   x.v_zero = false;
-  x.write_o = true;
+  x.out_mode = OUT_STORE;
   x.stop_on_zero = false;
-  x.lean = false;
+  x.gated = true;
   const size_t state_elems = (size_t)D * D;
   if (args.plan == PLAN_SEQ) {
     // CTAs start in index order; with seq_order the longest sequences go first, so
@@ -1600,31 +1622,35 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
     const int ns = args.n_seg;
     auto state_slot = [&](int s) { return args.seg_states + ((size_t)s * H + x.h) * state_elems; };
     int seg;
-    if (args.plan == PLAN_STATES) {
-      if (slot < ns - 2) {              // M_j, j = slot + 1
-        seg = slot + 1;
-        x.lean = true;
-        x.write_o = false;
+    if (args.plan == PLAN_ZERO) {
+      if (slot < ns) {                  // Z_j, j = slot
+        seg = slot;
+        x.h0 = (seg == 0 && args.h0) ? args.h0 + (size_t)x.h * state_elems : nullptr;
+        x.hT = state_slot(seg == ns - 1 ? 2 * ns - 3 : seg);
+        x.gated = seg == 0;   // (the others' outputs take their corrections first)
+      } else {                          // M_j, j = slot - n + 1
+        seg = slot - ns + 1;
+        x.gated = false;
+        x.out_mode = OUT_NONE;
         x.h0 = nullptr;
         x.h0_identity = true;
         x.v_zero = true;
         x.stop_on_zero = true;
         x.hT = state_slot(ns - 2 + seg);
-      } else if (slot < 2 * ns - 4) {   // R_j, j = slot - (n - 3)
-        seg = slot - (ns - 3);
-        x.lean = true;
-        x.write_o = false;
-        x.h0 = nullptr;
-        x.hT = state_slot(seg);
-      } else {                          // O_0
-        seg = 0;
-        x.h0 = args.h0 ? args.h0 + (size_t)x.h * state_elems : nullptr;
-        x.hT = state_slot(0);
       }
-    } else {
+    } else {                            // PLAN_CORR
       seg = slot + 1;
       x.h0 = state_slot(seg - 1);
-      x.hT = (seg == ns - 1 && args.hT) ? args.hT + (size_t)x.h * state_elems : nullptr;
+      x.gated = false;
+      x.v_zero = true;
+      x.stop_on_zero = true;
+      x.out_mode = OUT_ADD;
+      if (seg == ns - 1 && args.hT) {
+        x.hT = args.hT + (size_t)x.h * state_elems;
+        x.hT_base = state_slot(2 * ns - 3);
+      } else {
+        x.hT = nullptr;
+      }
     }
     auto seg_start = [&](int j) { return seg::seg_first_chunk(j, args.seg_base, args.seg_rem) * CHUNK; };
     x.bos = seg_start(seg);
@@ -1661,17 +1687,51 @@ kda_chunk_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_cons
   x.tmem = *tmem_slot;
 
   if (warp < PA_WARPS) {
-    prep_a_role<RT, MODE>(x, args);
+    prep_a_role<SPLIT, MODE>(x, args);
   } else if (warp < ST_WARP0) {
-    prep_b_role<RT, MODE>(x, &map_k, &map_q, &map_la);
+    prep_b_role<SPLIT, MODE>(x, &map_k, &map_q, &map_la);
   } else {
-    state_role<RT, MODE>(x, args, &map_v, &map_o);
+    state_role<SPLIT, MODE>(x, args, &map_v, &map_o);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == ST_WARP0) {
     tc_fence_after();
     tmem_dealloc(x.tmem, TM_COLS);
+  }
+}
+
+// ============================================================================
+// The fused variant's output of tokens [t0, t1) in a time split (segments 1 .. n-1,
+// whose raw outputs take their corrections first), in place, per (token, head) row of
+// 128 values: o <- o / sqrt(mean(o^2) + RMS_EPS) * norm_w * sigmoid(gate_pre), the
+// epilogue of the chunk kernel's gated CTAs. 16 threads per row, 16 bytes each; rows
+// are [row0, row0 + rows) of the [T*H][128] view.
+// ============================================================================
+constexpr int NG_THREADS = 256;
+constexpr int NG_ROWS = NG_THREADS / 16;   // rows per block and pass
+
+__global__ void __launch_bounds__(NG_THREADS)
+kda_norm_gate_kernel(__nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ gate_pre,
+                     const float* __restrict__ norm_w, int64_t row0, int64_t rows) {
+  const int sub = threadIdx.x & 15;
+  const unsigned mask = 0xFFFFu << (threadIdx.x & 16);   // this row's 16 lanes
+  float w8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w8[i] = __ldg(norm_w + 8 * sub + i);
+  const int64_t stride = (int64_t)gridDim.x * NG_ROWS;
+  for (int64_t r = (int64_t)blockIdx.x * NG_ROWS + (threadIdx.x >> 4); r < rows; r += stride) {
+    const size_t e = (size_t)(row0 + r) * D + 8 * sub;
+    const uint4 o8 = *reinterpret_cast<const uint4*>(o + e);
+    const uint4 g8 = ldg_nc_u4(gate_pre + e);
+    const uint32_t ov[4] = {o8.x, o8.y, o8.z, o8.w};
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ss += bf_lo(ov[i]) * bf_lo(ov[i]) + bf_hi(ov[i]) * bf_hi(ov[i]);
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(mask, ss, off);
+    const float inv = rsqrtf(ss * (1.f / D) + RMS_EPS);
+    *reinterpret_cast<uint4*>(o + e) = gate_row8(o8, g8, w8, inv);
   }
 }
 

@@ -3,9 +3,10 @@
 // Every step of the recurrence (Kimi Linear summary, section 3) is affine in the
 // state, so a segment of chunks maps its entering state S to M S + R, with M the
 // product of its per-token transitions (I - beta k k^T) Diag(alpha) and R its final
-// state from a zero start. The chunk kernel's state pass leaves, per head, the
-// exact state entering segment 1 in slot 0, R_j in slot j and M_j in slot n-2+j
-// (j = 1 .. n-2; M_j is the final state from the identity with v = 0). This kernel
+// state from a zero start. The chunk kernel's first pass of a split (PLAN_ZERO)
+// leaves, per head, the exact state entering segment 1 in slot 0, R_j in slot j and
+// M_j in slot n-2+j (j = 1 .. n-2; M_j is the final state from the identity with
+// v = 0). This kernel
 // then walks the segments in order,
 //     S_{j+1} = M_j S_j + R_j,   j = 1 .. n-2   (S_1 = slot 0),
 // writing S_{j+1} over R_j in slot j, all in fp32. One CTA per head; n-2 products
@@ -20,9 +21,6 @@ namespace seg {
 constexpr int SCAN_THREADS = 256;
 constexpr int SP = D + 4;   // smem pitch of the row-major copies (keeps float4 rows aligned)
 constexpr size_t SCAN_SMEM = 2 * (size_t)D * SP * sizeof(float);
-
-// Slots of the segment-state buffer [slots][H][128][128] (see the chunk kernel's plans).
-__host__ __device__ constexpr int slots(int n_seg) { return 2 * n_seg - 3; }
 
 // First chunk of segment j when n_chunks chunks are cut into n_seg segments balanced
 // to within one chunk: seg_base = n_chunks / n_seg, seg_rem = n_chunks % n_seg, and

@@ -104,21 +104,26 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_
  *
  * Every step of the recurrence is affine in the state, so a run of chunks maps
  * its entering state S to M S + R (M: product of the per-token transitions,
- * R: the final state from a zero start). With the time split the sequence is cut
- * into n >= 3 segments of whole chunks (balanced to within one chunk). A first
- * pass computes, in parallel, segment 0's output and final state and (R_j, M_j)
- * of the middle segments; the M_j runs stop early once their state is exactly
- * zero, which the erase and the decay bring about within a few hundred chunks on
- * typical inputs. A scan composes the maps into the state entering every segment,
- * and a second pass runs segments 1 .. n-1 in parallel from those states and
- * writes o and hT. n is chosen for the current device's SM count (see
- * kda_chunk_fwd_split_plan). The result is the same recurrence (exact in real
- * arithmetic; fp32 state throughout, bf16 MMA operands as in kda_chunk_fwd).
+ * R: the final state from a zero start), and its output is its output from a zero
+ * start plus that of the same run from S with v = 0. With the time split the
+ * sequence is cut into n >= 2 segments of whole chunks (balanced to within one
+ * chunk). A first pass runs every segment in parallel, segment 0 from h0 and the
+ * others from a zero state, storing their outputs and final states, together with
+ * the M_j of the middle segments (from the identity with v = 0). A scan composes
+ * the maps into the state entering every segment, and a second pass runs segments
+ * 1 .. n-1 from those states with v = 0, adding their outputs onto o, and sets hT.
+ * The M_j runs and the second pass stop once their state is exactly zero, which
+ * the erase and the decay bring about within some tens of chunks on typical
+ * inputs; without decay or erase they run to the ends of their segments. n is
+ * chosen for the current device's SM count (see kda_chunk_fwd_split_plan). The
+ * result is the same recurrence (exact in real arithmetic; fp32 state throughout,
+ * bf16 MMA operands as in kda_chunk_fwd; the outputs of segments 1 .. n-1 are
+ * rounded to bf16 twice, once per pass).
  *
  * Arguments: as kda_chunk_fwd, plus
  *   workspace        16-byte aligned device scratch, or NULL
  *   workspace_bytes  its size. The split takes the best plan whose scratch fits
- *                    ((2n - 3) * n_heads * 64 KiB); with NULL, or too little for
+ *                    ((2n - 2) * n_heads * 64 KiB); with NULL, or too little for
  *                    any split, the call is exactly kda_chunk_fwd (single pass).
  *                    kda_chunk_fwd_workspace_size(...) bytes give the best plan.
  * The workspace must stay untouched until the stream has passed the call.
@@ -139,7 +144,7 @@ int kda_chunk_fwd_ws(const void* q, const void* k, const void* v, const float* l
  * Returns the number of segments n (0: no split, the single pass runs), or a
  * negative kda_status (KDA_ERR_SHAPE for n_heads <= 0 or t_total < 0,
  * KDA_ERR_CUDA if n_sms is 0 and the device cannot be queried). If seg_bounds is
- * not NULL and n >= 3, it receives n + 1 token offsets: segment j covers tokens
+ * not NULL and n >= 2, it receives n + 1 token offsets: segment j covers tokens
  * [seg_bounds[j], seg_bounds[j+1]), seg_bounds[0] = 0, seg_bounds[n] = t_total,
  * every inner offset a multiple of 64, segments balanced to within one chunk, every
  * segment at least 16 chunks. At most KDA_MAX_SEGMENTS segments.
@@ -149,9 +154,11 @@ int kda_chunk_fwd_split_plan(int32_t n_heads, int64_t t_total, int32_t n_sms,
                              size_t workspace_bytes, int64_t* seg_bounds);
 
 /*
- * kda_chunk_fwd_workspace_size - bytes of workspace kda_chunk_fwd_ws would use for
- * these sizes on the current device (0: no time split applies). has_cu_seqlens is
- * nonzero when the call will pass a cu_seqlens array (then no split applies).
+ * kda_chunk_fwd_workspace_size - bytes of workspace that give kda_chunk_fwd_ws (and
+ * kda_gdn_chunk_fwd_ws, and for bf16 kda_chunk_fwd_fused, which split alike) their
+ * best time split for these sizes on the current device (0: no time split applies).
+ * has_cu_seqlens is nonzero when the call will pass a cu_seqlens array (then no split
+ * applies, and a packed batch of more CTAs than SMs uses 4 bytes per sequence).
  */
 size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_heads,
                                     kda_dtype qkv_dtype, int has_cu_seqlens);
@@ -171,8 +178,8 @@ size_t kda_chunk_fwd_workspace_size(int32_t n_seqs, int64_t t_total, int32_t n_h
  *
  * Scratch: one __device__ array of KDA_STATIC_SCRATCH_BYTES (16 MiB), 256-byte
  * aligned, in every GPU context that loads the library, held until the process
- * exits. The time split of one long sequence plans within it ((2n - 3) * n_heads
- * * 64 KiB for n segments: 14 MiB for 32 heads in 5 segments), so for a few head
+ * exits. The time split of one long sequence plans within it ((2n - 2) * n_heads
+ * * 64 KiB for n segments: 12 MiB for 32 heads in 4 segments), so for a few head
  * counts it splits into fewer segments than kda_chunk_fwd_ws given a workspace of
  * kda_chunk_fwd_workspace_size(...) bytes would. A packed batch of more CTAs than
  * SMs uses 4 bytes per sequence.
@@ -240,7 +247,12 @@ int kda_chunk_fwd_simt(const void* q, const void* k, const void* v, const float*
  *   gate_pre          [t_total, n_heads, 128] bf16
  *   norm_w            [128] fp32, shared by the heads
  *   h0, cu_seqlens, n_seqs, t_total, n_heads, hT, workspace, workspace_bytes:
- *                     as kda_chunk_fwd_ws (the same time split of one long sequence)
+ *                     as kda_chunk_fwd_ws, with the same time split of one long
+ *                     sequence. The gated output is not linear in the state, so in
+ *                     the split only segment 0's output is normalised and gated by
+ *                     the chunk kernel; segments 1 .. n-1 are stored raw, take their
+ *                     corrections, and a last pass over them (one more read and write
+ *                     of o, one read of gate_pre) applies the norm and the gate
  *   o                 [t_total, n_heads, 128] bf16, the gated output
  * t_total must be 0 or at least 64 (the tensor-core path); otherwise KDA_ERR_SHAPE.
  * Returns KDA_OK or a negative kda_status.

@@ -101,7 +101,6 @@ def test_fused_packed_batch_with_empty_and_short_sequences(kda):
 def test_fused_time_split(kda, x_mean):
     """32 heads split in 3 segments; with strong decay every chunk takes the exact path."""
     T, H = 64 * 60 + 9, 32
-    assert len(kda.split_plan(H, T)) - 1 == 3
     inp = kda_inputs.make_fused_prefill([T], H, x_mean=x_mean, seed=5, device="cuda")
     o, hT = _run(kda, inp)
     heads = [0, 13, 31]

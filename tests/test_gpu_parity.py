@@ -201,10 +201,11 @@ def test_time_split_32_heads_ragged(kda):
 
 
 def test_time_split_16_heads_mixed_decay(kda):
-    """16 heads split into 6 segments; strong-decay chunks put exact-path chunks into
-    every pass (the transition runs start from the identity with v = 0)."""
+    """16 heads split into 5 segments; strong-decay chunks put exact-path chunks into
+    every pass (the transition runs start from the identity with v = 0, the
+    corrections from the segments' entering states)."""
     T, H = 64 * 100 + 5, 16
-    assert _split_segments(kda, T, H) == 6
+    assert _split_segments(kda, T, H) == 5
     inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 3.0, True, seed=82,
                                   device="cuda")
     g = torch.Generator(device="cuda").manual_seed(83)
@@ -383,20 +384,20 @@ def test_nearly_parallel_keys_time_split(kda):
 
 
 def test_time_split_uneven_segments_4_heads(kda):
-    """4 heads over 321 chunks: 20 segments whose lengths differ by one chunk (the
-    chunk count is not a multiple of the segment count), plus a ragged tail."""
-    T, H = 321 * 64 + 13, 4
+    """4 heads over 321 chunks (the last one ragged): 17 segments whose lengths differ
+    by one chunk (the chunk count is not a multiple of the segment count)."""
+    T, H = 320 * 64 + 13, 4
     bounds = kda.split_plan(H, T)
-    assert len(bounds) - 1 == 20
+    assert len(bounds) - 1 == 17
     sizes = np.diff(bounds)
     assert bounds[0] == 0 and bounds[-1] == T and sizes.min() > 15 * 64   # >= 16 chunks
-    assert len(set(sizes[:-1].tolist())) == 2   # 17 and 16 chunks
+    assert len(set(sizes[:-1].tolist())) == 2   # 19 and 18 chunks
     inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 3.0, True, seed=86,
                                   device="cuda")
     o, hT = _run(kda, inp)
     o_ref, h_ref = _oracle(inp)
     e_o, e_s = rel_err(o, o_ref), rel_err(hT, h_ref)
-    print(f"4 heads, 20 segments: o {e_o:.2e} hT {e_s:.2e}")
+    print(f"4 heads, 17 segments: o {e_o:.2e} hT {e_s:.2e}")
     assert e_o <= TOL_BF16 and e_s <= TOL_BF16
     o_1, h_1 = _run(kda, inp, kernel="single")
     assert rel_err(o, o_1.double().cpu().numpy()) <= TOL_BF16
@@ -406,10 +407,11 @@ def test_time_split_uneven_segments_4_heads(kda):
 @pytest.mark.parametrize("x_mean", [0.0, -5.0])
 def test_time_split_transitions_vanish(kda, x_mean):
     """Strong decay (about -50 or -320 nats per chunk): every segment transition M_j
-    becomes exactly zero after a chunk or two, so its CTA stops early while the other
-    roles are still ahead of it. Results must match the oracle and the single pass."""
+    and every correction becomes exactly zero after a chunk or two, so its CTA stops
+    early while the other roles are still ahead of it. Results must match the oracle
+    and the single pass."""
     T, H = 64 * 100 + 5, 16
-    assert _split_segments(kda, T, H) == 6
+    assert _split_segments(kda, T, H) == 5
     inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, x_mean, True, seed=87,
                                   device="cuda")
     o, hT = _run(kda, inp)
@@ -421,17 +423,17 @@ def test_time_split_transitions_vanish(kda, x_mean):
     assert rel_err(o, o_1.double().cpu().numpy()) <= TOL_BF16
 
 
-def test_time_split_five_segments_long(kda):
-    """32 heads over 3000 chunks: 5 segments of 600 chunks, with the transition runs
-    expected to end early (the headline plan at a fifth of its length). The oracle
-    follows 3 heads end to end."""
+def test_time_split_long_segments(kda):
+    """32 heads over 3000 chunks: 4 segments of 750 chunks, with the transition runs
+    and the corrections expected to end early (the long-context plan at a fifth of
+    its length). The oracle follows 3 heads end to end."""
     T, H = 3000 * 64, 32
-    assert _split_segments(kda, T, H) == 5
+    assert _split_segments(kda, T, H) == 4
     inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 4.0, True, seed=88,
                                   device="cuda")
     o, hT = _run(kda, inp)
     heads = [0, 17, 31]
     o_ref, h_ref = _oracle(inp, heads)
     e_o, e_s = rel_err(o[:, heads], o_ref), rel_err(hT[:, heads], h_ref)
-    print(f"5 segments: o {e_o:.2e} hT {e_s:.2e}")
+    print(f"4 segments of 750 chunks: o {e_o:.2e} hT {e_s:.2e}")
     assert e_o <= TOL_BF16 and e_s <= TOL_BF16

@@ -10,8 +10,8 @@ multiple of the segment counts, a plan must
     and every inner bound is a whole chunk;
   * give every segment at least 16 chunks, with lengths differing by at most one chunk
     (the last segment alone may end in a partial chunk);
-  * fit one wave of SMs with its output pass: H (n - 1) <= SMs;
-  * fit the scratch it is given: (2n - 3) * H * 64 KiB.
+  * fit one wave of SMs with its segments: H n <= SMs;
+  * fit the scratch it is given: (2n - 2) * H * 64 KiB.
 """
 
 from __future__ import annotations
@@ -37,15 +37,15 @@ def lib():
 def _plan(lib, H, T, sms=SMS, ws=_native.SIZE_MAX):
     b = (ctypes.c_int64 * (_native.KDA_MAX_SEGMENTS + 1))()
     n = lib.kda_chunk_fwd_split_plan(H, T, sms, ws, b)
-    return n, [int(b[i]) for i in range(n + 1)] if n >= 3 else []
+    return n, [int(b[i]) for i in range(n + 1)] if n >= 2 else []
 
 
 def _check(H, T, n, bounds, sms, ws):
     if n == 0:
         return
-    assert 3 <= n <= _native.KDA_MAX_SEGMENTS
-    assert H * (n - 1) <= sms
-    assert (2 * n - 3) * H * SLOT <= ws
+    assert 2 <= n <= _native.KDA_MAX_SEGMENTS
+    assert H * n <= sms
+    assert (2 * n - 2) * H * SLOT <= ws
     assert bounds[0] == 0 and bounds[-1] == T
     b = np.array(bounds)
     assert np.all(np.diff(b) > 0)
@@ -65,22 +65,31 @@ def test_plan_covers_sequence(lib, H):
             assert n >= 0
             _check(H, T, n, bounds, SMS, _native.SIZE_MAX)
             seen.add(n)
-    if H <= SMS // 2:
+    if H <= SMS // 3:
         assert max(seen) >= 3   # some length splits
 
 
 def test_reported_case_4_heads_321_chunks(lib):
-    # 4 heads and 321 chunks: 20 segments of 17 and 16 chunks (no segment past the end)
+    # 4 heads and 321 chunks: 17 segments of 19 and 18 chunks (no segment past the end)
     n, bounds = _plan(lib, 4, 321 * 64)
-    assert n == 20
+    assert n == 17
     _check(4, 321 * 64, n, bounds, SMS, _native.SIZE_MAX)
+    assert sorted(set(np.diff(bounds).tolist())) == [18 * 64, 19 * 64]
 
 
 def test_headline_plan(lib):
-    # 32 heads, 1,048,576 tokens: 5 segments of 3276-3277 chunks
+    # 32 heads, 1,048,576 tokens: 4 segments of 4096 chunks (128 CTAs side by side)
     n, bounds = _plan(lib, 32, 1 << 20)
-    assert n == 5
-    assert np.diff(bounds).tolist() == [3277 * 64] * 4 + [3276 * 64]
+    assert n == 4
+    assert np.diff(bounds).tolist() == [4096 * 64] * 4
+
+
+def test_short_segments_plan_for_full_corrections(lib):
+    # 32 heads, 64 chunks: segments too short for the corrections to be counted on
+    # stopping early, so the plan weighs a full correction pass: 3 segments
+    assert _plan(lib, 32, 4096)[0] == 3
+    # 16 heads over 1M tokens: 9 segments (144 CTAs)
+    assert _plan(lib, 16, 1 << 20)[0] == 9
 
 
 def test_plan_fits_given_scratch(lib):
@@ -88,11 +97,12 @@ def test_plan_fits_given_scratch(lib):
         for ws in (0, 3 * H * SLOT, 16 << 20, _native.SIZE_MAX):
             n, bounds = _plan(lib, H, 1 << 20, ws=ws)
             _check(H, 1 << 20, n, bounds, SMS, ws)
-        assert _plan(lib, H, 1 << 20, ws=3 * H * SLOT - 1)[0] == 0   # below one split
+        assert _plan(lib, H, 1 << 20, ws=2 * H * SLOT - 1)[0] == 0   # below one split
 
 
 def test_short_and_fp32_cases_do_not_split(lib):
-    assert _plan(lib, 32, 64 * 47)[0] == 0      # fewer than 3 x 16 chunks
+    assert _plan(lib, 32, 64 * 31)[0] == 0      # fewer than 2 x 16 chunks
     assert _plan(lib, 32, 63)[0] == 0           # shorter than one chunk: CUDA-core kernel
     assert _plan(lib, 100, 1 << 20)[0] == 0     # 2 x 100 heads exceed one wave
+    assert _plan(lib, 32, 64 * 40)[0] == 0      # no split pays at 40 chunks
     assert lib.kda_chunk_fwd_split_plan(0, 100, SMS, 0, None) == _native.KDA_ERR_SHAPE

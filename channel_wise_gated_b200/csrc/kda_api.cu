@@ -119,20 +119,23 @@ bool encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 // Every segment keeps at least MIN_SEG_CHUNKS chunks; at most MAX_SEGMENTS.
 constexpr int MIN_SEG_CHUNKS = 16;
 constexpr int MAX_SEGMENTS = 64;
-constexpr int64_t SPLIT_EARLY_CHUNKS = 512;
+constexpr int64_t SPLIT_EARLY_CHUNKS = 128;
 
 // Time split of one long sequence (the chunk kernel's PLAN_ZERO, the segment scan,
-// PLAN_CORR; see the kernel's plans). A split into n segments runs all n segments from
-// zero states side by side (H n CTAs, which must fit one wave), the n - 2 transition
-// chains per head on the SMs left over or after them, the scan (n - 2 products of
-// 128 x 128 matrices per head, about two chunk periods each), and n - 1
-// corrections per head. Transition chains and corrections both stop once their
-// state is exactly zero; for segments of SPLIT_EARLY_CHUNKS chunks or more the plan
-// counts on that within STOP_CHUNKS chunks, and otherwise on neither stopping. In
-// chunk periods a split costs one segment, plus the transition chains that do not
-// fit beside the segments, plus the scan, plus one correction; the single pass
-// costs the whole sequence. Every segment keeps at least MIN_SEG_CHUNKS chunks, and
-// the plan's scratch must fit the bytes available.
+// PLAN_CORR; see the kernel's plans). A split into n segments of about len chunks runs
+// the H n Z CTAs (all segments from zero states) in waves of one CTA per SM; the SMs
+// the last wave leaves free take the H (n - 2) transition chains, the rest follow the
+// Z CTAs. Then the scan (n - 2 products of 128 x 128 matrices per head, about two
+// chunk periods each) and the H (n - 1) corrections. Transition chains and
+// corrections both stop once their state is exactly zero; for segments of
+// SPLIT_EARLY_CHUNKS chunks or more the plan counts on that within STOP_CHUNKS
+// chunks, and otherwise on neither stopping. In chunk periods a split costs
+//   waves(H n) len + (transition chains that do not fit) + 2 (n - 2) + waves(H (n - 1)) z
+// and the single pass the whole sequence. Equal segments make the waves even: at 32
+// heads over 1M tokens, 9 segments (two waves of 148 and 140 Z CTAs) measured 18.1 ms
+// against 19.6 ms for 4 (one wave of 128), 20.0 for 8 and 23.5 for 10 (three waves).
+// Every segment keeps at least MIN_SEG_CHUNKS chunks, and the plan's scratch must fit
+// the bytes available.
 constexpr int64_t STOP_CHUNKS = 64;
 constexpr double SCAN_STEP_CHUNKS = 2.0;
 
@@ -146,15 +149,15 @@ int split_segments(int64_t n_chunks, int32_t n_heads, int sms, size_t max_bytes)
   double best_cost = (double)n_chunks * (double)((n_heads + sms - 1) / sms);
   for (int n = 2; n <= MAX_SEGMENTS; ++n) {
     if (n_chunks < (int64_t)n * MIN_SEG_CHUNKS) break;
-    if ((int64_t)n_heads * n > sms) break;
     if (split_workspace_bytes(n, n_heads) > max_bytes) break;
-    const double len = (double)((n_chunks + n - 1) / n);
-    const double z = len >= (double)SPLIT_EARLY_CHUNKS ? std::min(len, (double)STOP_CHUNKS) : len;
-    const int64_t trans = (int64_t)n_heads * (n - 2), spare = sms - (int64_t)n_heads * n;
-    double extra = 0.0;
-    if (trans > 0 && (spare == 0 || (double)((trans + spare - 1) / spare) * z > len))
-      extra = z * (double)((trans + sms - 1) / sms);
-    const double cost = len + extra + SCAN_STEP_CHUNKS * (n - 2) + z;
+    const int64_t len = (n_chunks + n - 1) / n;
+    const double z = len >= SPLIT_EARLY_CHUNKS ? (double)std::min<int64_t>(len, STOP_CHUNKS) : (double)len;
+    const int64_t zc = (int64_t)n_heads * n, waves = (zc + sms - 1) / sms;
+    const int64_t trans = (int64_t)n_heads * (n - 2), free_sms = waves * sms - zc;
+    const int64_t fit = free_sms * std::max<int64_t>(1, (int64_t)((double)len / z));
+    const double extra = trans > fit ? z * (double)((trans - fit + sms - 1) / sms) : 0.0;
+    const int64_t cwaves = ((int64_t)n_heads * (n - 1) + sms - 1) / sms;
+    const double cost = (double)(waves * len) + extra + SCAN_STEP_CHUNKS * (n - 2) + (double)cwaves * z;
     if (cost < best_cost - 1e-9) {
       best_cost = cost;
       best = n;

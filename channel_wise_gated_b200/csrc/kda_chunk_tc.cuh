@@ -1216,11 +1216,11 @@ __device__ __forceinline__ void tile_rows_out(const uint8_t* dt, __nv_bfloat16* 
     __nv_bfloat16* g = orow + (size_t)r * rs + 8 * seg;
     if (!add) {
       *reinterpret_cast<uint4*>(g) = v;
-    } else {
+    } else {   // (reductions: nothing waits for their results)
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        atomicAdd(reinterpret_cast<__nv_bfloat162*>(g) + k, *reinterpret_cast<const __nv_bfloat162*>(&w4[k]));
+        asm volatile("red.global.add.noftz.bf16x2 [%0], %1;" ::"l"(g + 2 * k), "r"(w4[k]) : "memory");
     }
   }
 }

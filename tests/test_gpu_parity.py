@@ -423,6 +423,20 @@ def test_time_split_transitions_vanish(kda, x_mean):
     assert rel_err(o, o_1.double().cpu().numpy()) <= TOL_BF16
 
 
+def test_time_split_two_segments(kda):
+    """48 heads over 256 chunks: 2 segments (no transition chain, no scan: the correction
+    starts from segment 0's final state), ragged tail, random h0."""
+    T, H = 256 * 64 - 21, 48
+    assert _split_segments(kda, T, H) == 2
+    inp = kda_inputs.make_prefill([T], H, torch.bfloat16, torch.float32, 3.0, True, seed=89,
+                                  device="cuda")
+    o, hT = _run(kda, inp)
+    o_ref, h_ref = _oracle(inp)
+    e_o, e_s = rel_err(o, o_ref), rel_err(hT, h_ref)
+    print(f"2 segments: o {e_o:.2e} hT {e_s:.2e}")
+    assert e_o <= TOL_BF16 and e_s <= TOL_BF16
+
+
 def test_time_split_long_segments(kda):
     """32 heads over 3000 chunks: 4 segments of 750 chunks, with the transition runs
     and the corrections expected to end early (the long-context plan at a fifth of

@@ -246,15 +246,20 @@ struct Ctx {
 constexpr int ABORT_TIMEOUT = 1, ABORT_DONE = 2;
 
 // Bounded per-thread wait that also gives up when another role aborted. The
-// thread sleeps in the barrier (suspend hint) instead of spinning. (Out of line,
-// with scalar arguments only, so that callers keep their context in registers.)
-// (The bound lives in shared memory beside the abort word: MISC_WAIT_NS.)
+// thread sleeps in the barrier (suspend hint) instead of spinning, and looks at the
+// abort word at least every WAKE_NS: a chain that stops early (ABORT_DONE) leaves its
+// other roles blocked on barriers that will not complete, and the CTA holds its SM
+// until they notice (with a 200 us hint, a correction pass of 2 segments took 0.51
+// ms where its CTAs' work took 0.30). (Out of line, with scalar arguments only, so
+// that callers keep their context in registers. The bound lives in shared memory
+// beside the abort word: MISC_WAIT_NS.)
+constexpr uint32_t WAKE_NS = 2000;
 __device__ __noinline__ bool wait_b_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const uint64_t t0 = globaltimer_ns();
   const uint64_t limit = *reinterpret_cast<const volatile uint64_t*>(
       reinterpret_cast<volatile uint8_t*>(abort_flag) + MISC_WAIT_NS);
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (mbar_try_wait_sleep(bar, parity, WAKE_NS)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > limit) {
       *abort_flag = ABORT_TIMEOUT;

@@ -10,7 +10,8 @@
 // then walks the segments in order,
 //     S_{j+1} = M_j S_j + R_j,   j = 1 .. n-2   (S_1 = slot 0),
 // writing S_{j+1} over R_j in slot j, all in fp32. One CTA per head; n-2 products
-// of 128 x 128 matrices, a few microseconds in all.
+// of 128 x 128 matrices, about 20 us each. A transition chain that stopped early
+// left M_j exactly zero: then S_{j+1} = R_j, already in place, and the step is skipped.
 #pragma once
 
 #include "kda_common.cuh"
@@ -44,12 +45,15 @@ kda_segment_scan_kernel(float* __restrict__ states, int n_heads, int n_seg) {
     const float* M = slot(n_seg - 2 + j);       // M_j
     const float* S = slot(j - 1);               // S_j (slot 0, or the previous result)
     float* RS = slot(j);                        // R_j in, S_{j+1} out
+    int nz = 0;
     for (int i = tid; i < D * D / 4; i += SCAN_THREADS) {
       const int r = (4 * i) / D, c = (4 * i) % D;
-      *reinterpret_cast<float4*>(&Ms[r * SP + c]) = reinterpret_cast<const float4*>(M)[i];
+      const float4 m4 = reinterpret_cast<const float4*>(M)[i];
+      nz |= (m4.x != 0.f) | (m4.y != 0.f) | (m4.z != 0.f) | (m4.w != 0.f);
+      *reinterpret_cast<float4*>(&Ms[r * SP + c]) = m4;
       *reinterpret_cast<float4*>(&Ss[r * SP + c]) = reinterpret_cast<const float4*>(S)[i];
     }
-    __syncthreads();
+    if (!__syncthreads_or(nz)) continue;   // M_j = 0: S_{j+1} = R_j (the loop's barrier is passed)
     float acc[8][8];
 #pragma unroll
     for (int a = 0; a < 8; ++a)

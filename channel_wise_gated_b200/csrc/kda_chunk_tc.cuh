@@ -1210,23 +1210,14 @@ __device__ __forceinline__ void st_store_state(uint32_t lane_addr, float* hT, co
 }
 // The valid rows (< L) of the staged output tile ([64 rows][128 columns] bf16 in two
 // 64-column halves of 8 KB, 128B-swizzled rows) to o at orow (the chunk's first row,
-// the head's first column): stored, or added onto what is there (bf16x2 atomic adds,
-// for a correction). 16 bytes (8 columns) per step, all state threads.
+// the head's first column). 16 bytes (8 columns) per step, all state threads.
 __device__ __forceinline__ void tile_rows_out(const uint8_t* dt, __nv_bfloat16* orow, size_t rs, int L,
-                                              bool add, int tid) {
+                                              int tid) {
 #pragma unroll 1
   for (int i = tid; i < L * 16; i += ST_THREADS) {
     const int r = i >> 4, seg = i & 15;
-    const uint4 v = *reinterpret_cast<const uint4*>(dt + (seg >> 3) * 8192 + swz128(r * 128 + (seg & 7) * 16));
-    __nv_bfloat16* g = orow + (size_t)r * rs + 8 * seg;
-    if (!add) {
-      *reinterpret_cast<uint4*>(g) = v;
-    } else {   // (reductions: nothing waits for their results)
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        asm volatile("red.global.add.noftz.bf16x2 [%0], %1;" ::"l"(g + 2 * k), "r"(w4[k]) : "memory");
-    }
+    *reinterpret_cast<uint4*>(orow + (size_t)r * rs + 8 * seg) =
+        *reinterpret_cast<const uint4*>(dt + (seg >> 3) * 8192 + swz128(r * 128 + (seg & 7) * 16));
   }
 }
 
@@ -1476,10 +1467,12 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       const int64_t t0 = x.bos + (int64_t)co * CHUNK;
       const int L = (x.eos - t0) < CHUNK ? (int)(x.eos - t0) : CHUNK;
       // The output goes through the output tile (its previous store has read it): a full
-      // chunk to be stored leaves by one TMA store of [64 rows][128 columns], a ragged last
-      // chunk or a correction by a short loop over its valid rows.
+      // chunk to be stored leaves by one TMA store of [64 rows][128 columns], a correction
+      // by one TMA reduce-add (its chunks are whole but for the very last of the tensor,
+      // whose rows past the end the copy clips), and a ragged last chunk of a sequence by a
+      // short loop over its valid rows.
       const bool staged = omode != OUT_NONE;
-      const bool tile_out = staged && L == CHUNK && omode == OUT_STORE;
+      const bool tile_out = (omode == OUT_STORE && L == CHUNK) || omode == OUT_ADD;
       alive = alive && wait_b(x, B_PD, co & 1);
       if (alive) {
         tc_fence_after();
@@ -1494,7 +1487,7 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
       }
       if (staged && !tile_out) {
         named_bar_sync(BAR_OUT, ST_THREADS);
-        if (alive) tile_rows_out(dt, p.o + (size_t)t0 * x.rs + x.h * D, x.rs, L, omode == OUT_ADD, tid);
+        if (alive) tile_rows_out(dt, p.o + (size_t)t0 * x.rs + x.h * D, x.rs, L, tid);
         named_bar_sync(BAR_OUT, ST_THREADS);   // (before the tile is staged again)
       }
       if (tile_out) {
@@ -1505,8 +1498,13 @@ __device__ void state_role(const Ctx& x, const Args& p, const CUtensorMap* map_v
         } else {
           named_bar_sync(BAR_OUT, ST_THREADS);
           if (issuer && alive) {
-            tma_store_2d(map_o, dt, x.h * D, (int)t0);
-            tma_store_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);
+            if (omode == OUT_ADD) {
+              tma_reduce_add_2d(map_o, dt, x.h * D, (int)t0);
+              tma_reduce_add_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);
+            } else {
+              tma_store_2d(map_o, dt, x.h * D, (int)t0);
+              tma_store_2d(map_o, dt + 8192, x.h * D + 64, (int)t0);
+            }
             bulk_commit_group();
           }
         }

@@ -155,6 +155,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                "r"(smem_u32(src_smem)), "r"(x), "r"(y)
                : "memory");
 }
+// The same tile added onto global memory (element type from the tensor map; rows past
+// the tensor's end are clipped, as for the store)
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src_smem, int32_t x,
+                                                  int32_t y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src_smem)), "r"(x), "r"(y)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -128,8 +128,9 @@ constexpr int DEC_MAX_TOKENS = 16;
 // Shared memory of the multi-token step (dynamic: more than the 48 KB of static data).
 struct DecTokensSmem {
   float k[DEC_MAX_TOKENS][D], q[DEC_MAX_TOKENS][D], a[DEC_MAX_TOKENS][D], v[DEC_MAX_TOKENS][D];
-  // the partial projections, double-buffered by token parity: one barrier per token
+  // the partial projections and the reduced delta, double-buffered by token parity
   float4 u[2][DEC_THREADS / 32][32], y[2][DEC_THREADS / 32][32];
+  float dl[2][D];
   float beta[DEC_MAX_TOKENS], kq[DEC_MAX_TOKENS];
 };
 
@@ -172,8 +173,8 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
     s_a[t][c] = expf(to_f32(log_alpha[base]));
   }
   if (tid < n_tokens) s_beta[tid] = to_f32(beta[((size_t)seq * n_tokens + tid) * n_heads + h]);
-  // this lane's 4 output columns of token 0; one token further is n_heads * D elements
-  TQ* od = o + ((size_t)seq * n_tokens * n_heads + h) * D + lane * 4;
+  // the output row of token 0; one token further is n_heads * D elements
+  TQ* od = o + ((size_t)seq * n_tokens * n_heads + h) * D;
   const size_t o_step = (size_t)n_heads * D;
   __syncthreads();
   // k^T q of every token once (warp w takes tokens w, w + 8), formed exactly as the
@@ -215,30 +216,26 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
     }
     s_u[buf][warp][lane] = u;
     s_y[buf][warp][lane] = y;
-    // (this token's buffer was last read two tokens ago, before the previous barrier)
+    // (this token's buffers were last read two tokens ago, before the previous barriers)
     __syncthreads();
 
-    u = make_float4(0.f, 0.f, 0.f, 0.f);
-    y = make_float4(0.f, 0.f, 0.f, 0.f);
+    // thread c < 128 reduces column c over the warps, in the single step's order, and
+    // leaves delta_c for all; the other threads wait at the next barrier. (Each thread
+    // summing its own 4 columns, as the single step does, reads 8x the shared memory.)
+    if (tid < D) {
+      const int cl = tid >> 2, cc = tid & 3;
+      float uc = 0.f, yc = 0.f;
 #pragma unroll
-    for (int w = 0; w < DEC_THREADS / 32; ++w) {
-      const float4 a = s_u[buf][w][lane], b = s_y[buf][w][lane];
-      u.x += a.x; u.y += a.y; u.z += a.z; u.w += a.w;
-      y.x += b.x; y.y += b.y; y.z += b.z; y.w += b.w;
+      for (int w = 0; w < DEC_THREADS / 32; ++w) {
+        uc += reinterpret_cast<const float*>(&s_u[buf][w][cl])[cc];
+        yc += reinterpret_cast<const float*>(&s_y[buf][w][cl])[cc];
+      }
+      const float dc = s_beta[t] * (s_v[t][tid] - uc);
+      sm.dl[buf][tid] = dc;
+      od[tid] = from_f32<TQ>(fmaf(s_kq[t], dc, yc));
     }
-    const float kq = s_kq[t];
-    const float bt = s_beta[t];
-    const float4 vv = reinterpret_cast<const float4*>(s_v[t])[lane];
-    float4 dl;
-    dl.x = bt * (vv.x - u.x); dl.y = bt * (vv.y - u.y);
-    dl.z = bt * (vv.z - u.z); dl.w = bt * (vv.w - u.w);
-
-    if (warp == 0) {
-      od[0] = from_f32<TQ>(fmaf(kq, dl.x, y.x));
-      od[1] = from_f32<TQ>(fmaf(kq, dl.y, y.y));
-      od[2] = from_f32<TQ>(fmaf(kq, dl.z, y.z));
-      od[3] = from_f32<TQ>(fmaf(kq, dl.w, y.w));
-    }
+    __syncthreads();
+    const float4 dl = reinterpret_cast<const float4*>(sm.dl[buf])[lane];
 #pragma unroll
     for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
       const float4 k4 = *reinterpret_cast<const float4*>(&s_k[t][row0 + i4]);

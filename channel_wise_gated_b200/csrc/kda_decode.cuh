@@ -18,6 +18,7 @@
 #pragma once
 
 #include "kda_common.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
 
@@ -121,150 +122,201 @@ namespace kda {
 // is the single step's above, in the same order, so the result equals n_tokens
 // consecutive single steps. Inputs are packed sequence-major like a prefill batch of
 // equal lengths: [n_seqs, n_tokens, n_heads, 128] (beta [n_seqs, n_tokens, n_heads]).
-// All tokens' inputs are staged in shared memory up front, their loads in flight
-// together with the state's.
+//
+// Two persistent CTAs per SM each walk the states blockIdx.x, + gridDim.x, ... While a
+// CTA computes the tokens of one state from registers, a bulk copy brings the next state
+// into a 64 KB shared-memory buffer, so its load no longer sits between two states. (Per
+// CTA the load had taken 3.7 of a state's 7.5 us, with no other work to hide it.)
 constexpr int DEC_MAX_TOKENS = 16;
+constexpr uint32_t DEC_STATE_BYTES = D * D * sizeof(float);   // 64 KiB
 
-// Shared memory of the multi-token step (dynamic: more than the 48 KB of static data).
-struct DecTokensSmem {
-  float k[DEC_MAX_TOKENS][D], q[DEC_MAX_TOKENS][D], a[DEC_MAX_TOKENS][D], v[DEC_MAX_TOKENS][D];
-  // the partial projections and the reduced delta, double-buffered by token parity
-  float4 u[2][DEC_THREADS / 32][32], y[2][DEC_THREADS / 32][32];
-  float dl[2][D];
-  float beta[DEC_MAX_TOKENS], kq[DEC_MAX_TOKENS];
-};
+// Untiled bulk copy global -> shared (both addresses 16-byte aligned, bytes a multiple
+// of 16), completing `bytes` of the barrier's transaction count. No multicast.
+__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   sm100::smem_u32(dst_smem)),
+               "l"(src), "r"(bytes), "r"(sm100::smem_u32(bar))
+               : "memory");
+}
+
+// Dynamic shared memory of the multi-token step, in bytes, for n_tokens tokens: the state
+// buffer, its barrier, the tokens' k, q, alpha, v in fp32, the partial projections and the
+// reduced delta double-buffered by token parity, beta and k.q.
+__host__ __device__ constexpr size_t dec_tokens_smem_bytes(int n_tokens) {
+  return DEC_STATE_BYTES + 16 + (size_t)4 * n_tokens * D * sizeof(float) +
+         2 * 2 * (DEC_THREADS / 32) * 32 * sizeof(float4) + 2 * D * sizeof(float) +
+         2 * DEC_MAX_TOKENS * sizeof(float);
+}
 
 template <typename TQ, typename TG>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
 kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
                          const TQ* __restrict__ v, const TG* __restrict__ log_alpha,
                          const TG* __restrict__ beta, float* __restrict__ state,
-                         TQ* __restrict__ o, int n_heads, int n_tokens) {
-  const int chain = blockIdx.x;          // (sequence, head) flattened, as the state
-  const int seq = chain / n_heads, h = chain - seq * n_heads;
+                         TQ* __restrict__ o, int n_heads, int n_tokens, int n_chains) {
+  using namespace sm100;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  extern __shared__ __align__(16) unsigned char dec_smem[];
-  DecTokensSmem& sm = *reinterpret_cast<DecTokensSmem*>(dec_smem);
-  auto& s_k = sm.k;
-  auto& s_q = sm.q;
-  auto& s_a = sm.a;
-  auto& s_v = sm.v;
-  auto& s_u = sm.u;
-  auto& s_y = sm.y;
-  auto& s_beta = sm.beta;
-  auto& s_kq = sm.kq;
-
-  float4* S = reinterpret_cast<float4*>(state + (size_t)chain * D * D);
+  extern __shared__ __align__(128) unsigned char dec_smem[];
+  const float4* sbuf = reinterpret_cast<const float4*>(dec_smem);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(dec_smem + DEC_STATE_BYTES);
+  float* s_k = reinterpret_cast<float*>(dec_smem + DEC_STATE_BYTES + 16);   // [n_tokens][D]
+  float* s_q = s_k + n_tokens * D;
+  float* s_a = s_q + n_tokens * D;
+  float* s_v = s_a + n_tokens * D;
+  float4 (*s_u)[DEC_THREADS / 32][32] = reinterpret_cast<float4 (*)[DEC_THREADS / 32][32]>(s_v + n_tokens * D);
+  float4 (*s_y)[DEC_THREADS / 32][32] = s_u + 2;
+  float (*s_dl)[D] = reinterpret_cast<float (*)[D]>(s_y + 2);
+  float* s_beta = reinterpret_cast<float*>(s_dl + 2);
+  float* s_kq = s_beta + DEC_MAX_TOKENS;
   const int row0 = warp * DEC_ROWS_PER_WARP;
 
-  float4 s[DEC_ROWS_PER_WARP];
-#pragma unroll
-  for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) s[i] = __ldcs(&S[(row0 + i) * (D / 4) + lane]);
-
-#pragma unroll 1
-  for (int i = tid; i < n_tokens * D; i += DEC_THREADS) {
-    const int t = i / D, c = i - t * D;
-    const size_t base = (((size_t)seq * n_tokens + t) * n_heads + h) * D + c;
-    s_k[t][c] = to_f32(k[base]);
-    s_q[t][c] = to_f32(q[base]);
-    s_v[t][c] = to_f32(v[base]);
-    s_a[t][c] = expf(to_f32(log_alpha[base]));
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
   }
-  if (tid < n_tokens) s_beta[tid] = to_f32(beta[((size_t)seq * n_tokens + tid) * n_heads + h]);
-  // the output row of token 0; one token further is n_heads * D elements
-  TQ* od = o + ((size_t)seq * n_tokens * n_heads + h) * D;
-  const size_t o_step = (size_t)n_heads * D;
   __syncthreads();
-  // k^T q of every token once (warp w takes tokens w, w + 8), formed exactly as the
-  // single step forms it; read after the first token's barrier
-#pragma unroll 1
-  for (int t = warp; t < n_tokens; t += DEC_THREADS / 32) {
-    float kq = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) kq = fmaf(s_k[t][lane * 4 + i], s_q[t][lane * 4 + i], kq);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-    if (lane == 0) s_kq[t] = kq;
+  int chain = blockIdx.x;          // (sequence, head) flattened, as the state
+  if (tid == 0 && chain < n_chains) {
+    mbar_arrive_expect_tx(bar, DEC_STATE_BYTES);
+    bulk_load(dec_smem, state + (size_t)chain * D * D, DEC_STATE_BYTES, bar);
   }
+  uint32_t phase = 0;
+#pragma unroll 1
+  for (; chain < n_chains; chain += gridDim.x) {
+    const int seq = chain / n_heads, h = chain - seq * n_heads;
+#pragma unroll 1
+    for (int i = tid; i < n_tokens * D; i += DEC_THREADS) {
+      const int t = i / D, c = i - t * D;
+      const size_t base = (((size_t)seq * n_tokens + t) * n_heads + h) * D + c;
+      s_k[i] = to_f32(k[base]);
+      s_q[i] = to_f32(q[base]);
+      s_v[i] = to_f32(v[base]);
+      s_a[i] = expf(to_f32(log_alpha[base]));
+    }
+    if (tid < n_tokens) s_beta[tid] = to_f32(beta[((size_t)seq * n_tokens + tid) * n_heads + h]);
+    // this chain's state, copied into the buffer while the previous chain computed
+    const bool landed = mbar_wait(bar, phase);
+    phase ^= 1u;
+    float4 s[DEC_ROWS_PER_WARP];
+#pragma unroll
+    for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) s[i] = sbuf[(row0 + i) * (D / 4) + lane];
+    fence_proxy_async_smem();   // (these reads come before the next copy into the buffer)
+    if (!__syncthreads_and(landed)) {   // (also the barrier before the staged inputs are read)
+      if (tid == 0) {
+        flag_error(DEVERR_TIMEOUT);
+        mbar_wait(bar, phase ^ 1u, 100000000ull);   // (never leave with the copy in flight)
+      }
+      break;
+    }
+    if (tid == 0 && chain + (int)gridDim.x < n_chains) {
+      mbar_arrive_expect_tx(bar, DEC_STATE_BYTES);
+      bulk_load(dec_smem, state + (size_t)(chain + gridDim.x) * D * D, DEC_STATE_BYTES, bar);
+    }
+    float4* S = reinterpret_cast<float4*>(state + (size_t)chain * D * D);
+    // the output row of token 0; one token further is n_heads * D elements
+    TQ* od = o + ((size_t)seq * n_tokens * n_heads + h) * D;
+    const size_t o_step = (size_t)n_heads * D;
+    // k^T q of every token once (warp w takes tokens w, w + 8), formed exactly as the
+    // single step forms it; read after the first token's barrier
+#pragma unroll 1
+    for (int t = warp; t < n_tokens; t += DEC_THREADS / 32) {
+      float kq = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) kq = fmaf(s_k[t * D + lane * 4 + i], s_q[t * D + lane * 4 + i], kq);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+      if (lane == 0) s_kq[t] = kq;
+    }
 
 #pragma unroll 1
-  for (int t = 0; t < n_tokens; ++t, od += o_step) {
-    const int buf = t & 1;
-    // decay and the two partial projections over this warp's rows (4 rows of the
-    // gates and keys per 16-byte read; rows in the single step's order)
-    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int t = 0; t < n_tokens; ++t, od += o_step) {
+      const int buf = t & 1;
+      const float* sa_t = s_a + t * D;
+      const float* sk_t = s_k + t * D;
+      const float* sq_t = s_q + t * D;
+      // decay and the two partial projections over this warp's rows (4 rows of the
+      // gates and keys per 16-byte read; rows in the single step's order)
+      float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
-      const float4 a4 = *reinterpret_cast<const float4*>(&s_a[t][row0 + i4]);
-      const float4 k4 = *reinterpret_cast<const float4*>(&s_k[t][row0 + i4]);
-      const float4 q4 = *reinterpret_cast<const float4*>(&s_q[t][row0 + i4]);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w},
-                  qv[4] = {q4.x, q4.y, q4.z, q4.w};
+      for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(&sa_t[row0 + i4]);
+        const float4 k4 = *reinterpret_cast<const float4*>(&sk_t[row0 + i4]);
+        const float4 q4 = *reinterpret_cast<const float4*>(&sq_t[row0 + i4]);
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w}, kv[4] = {k4.x, k4.y, k4.z, k4.w},
+                    qv[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i4 + e;
-        const float a = av[e], kr = kv[e], qr = qv[e];
-        s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
-        u.x = fmaf(kr, s[i].x, u.x); u.y = fmaf(kr, s[i].y, u.y);
-        u.z = fmaf(kr, s[i].z, u.z); u.w = fmaf(kr, s[i].w, u.w);
-        y.x = fmaf(qr, s[i].x, y.x); y.y = fmaf(qr, s[i].y, y.y);
-        y.z = fmaf(qr, s[i].z, y.z); y.w = fmaf(qr, s[i].w, y.w);
+        for (int e = 0; e < 4; ++e) {
+          const int i = i4 + e;
+          const float a = av[e], kr = kv[e], qr = qv[e];
+          s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+          u.x = fmaf(kr, s[i].x, u.x); u.y = fmaf(kr, s[i].y, u.y);
+          u.z = fmaf(kr, s[i].z, u.z); u.w = fmaf(kr, s[i].w, u.w);
+          y.x = fmaf(qr, s[i].x, y.x); y.y = fmaf(qr, s[i].y, y.y);
+          y.z = fmaf(qr, s[i].z, y.z); y.w = fmaf(qr, s[i].w, y.w);
+        }
       }
-    }
-    s_u[buf][warp][lane] = u;
-    s_y[buf][warp][lane] = y;
-    // (this token's buffers were last read two tokens ago, before the previous barriers)
-    __syncthreads();
+      s_u[buf][warp][lane] = u;
+      s_y[buf][warp][lane] = y;
+      // (this token's buffers were last read two tokens ago, before the previous barriers)
+      __syncthreads();
 
-    // thread c < 128 reduces column c over the warps, in the single step's order, and
-    // leaves delta_c for all; the other threads wait at the next barrier. (Each thread
-    // summing its own 4 columns, as the single step does, reads 8x the shared memory.)
-    if (tid < D) {
-      const int cl = tid >> 2, cc = tid & 3;
-      float uc = 0.f, yc = 0.f;
+      // thread c < 128 reduces column c over the warps, in the single step's order, and
+      // leaves delta_c for all; the other threads wait at the next barrier. (Each thread
+      // summing its own 4 columns, as the single step does, reads 8x the shared memory.)
+      if (tid < D) {
+        const int cl = tid >> 2, cc = tid & 3;
+        float uc = 0.f, yc = 0.f;
 #pragma unroll
-      for (int w = 0; w < DEC_THREADS / 32; ++w) {
-        uc += reinterpret_cast<const float*>(&s_u[buf][w][cl])[cc];
-        yc += reinterpret_cast<const float*>(&s_y[buf][w][cl])[cc];
+        for (int w = 0; w < DEC_THREADS / 32; ++w) {
+          uc += reinterpret_cast<const float*>(&s_u[buf][w][cl])[cc];
+          yc += reinterpret_cast<const float*>(&s_y[buf][w][cl])[cc];
+        }
+        const float dc = s_beta[t] * (s_v[t * D + tid] - uc);
+        s_dl[buf][tid] = dc;
+        od[tid] = from_f32<TQ>(fmaf(s_kq[t], dc, yc));
       }
-      const float dc = s_beta[t] * (s_v[t][tid] - uc);
-      sm.dl[buf][tid] = dc;
-      od[tid] = from_f32<TQ>(fmaf(s_kq[t], dc, yc));
-    }
-    __syncthreads();
-    const float4 dl = reinterpret_cast<const float4*>(sm.dl[buf])[lane];
+      __syncthreads();
+      const float4 dl = reinterpret_cast<const float4*>(s_dl[buf])[lane];
 #pragma unroll
-    for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
-      const float4 k4 = *reinterpret_cast<const float4*>(&s_k[t][row0 + i4]);
-      const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
+      for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
+        const float4 k4 = *reinterpret_cast<const float4*>(&sk_t[row0 + i4]);
+        const float kv[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = i4 + e;
-        const float kr = kv[e];
-        s[i].x = fmaf(kr, dl.x, s[i].x); s[i].y = fmaf(kr, dl.y, s[i].y);
-        s[i].z = fmaf(kr, dl.z, s[i].z); s[i].w = fmaf(kr, dl.w, s[i].w);
+        for (int e = 0; e < 4; ++e) {
+          const int i = i4 + e;
+          const float kr = kv[e];
+          s[i].x = fmaf(kr, dl.x, s[i].x); s[i].y = fmaf(kr, dl.y, s[i].y);
+          s[i].z = fmaf(kr, dl.z, s[i].z); s[i].w = fmaf(kr, dl.w, s[i].w);
+        }
       }
     }
+#pragma unroll
+    for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) __stcs(&S[(row0 + i) * (D / 4) + lane], s[i]);
+    __syncthreads();   // (the staged inputs are rewritten for the next chain)
   }
-#pragma unroll
-  for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) __stcs(&S[(row0 + i) * (D / 4) + lane], s[i]);
 }
 
-// Host side: one CTA per (sequence, head); returns the launch's CUDA error.
+// Host side: two persistent CTAs per SM (or one per state, if fewer); returns the
+// launch's CUDA error.
 template <typename TQ, typename TG>
 cudaError_t launch_decode_tokens(const TQ* q, const TQ* k, const TQ* v, const TG* log_alpha,
                                  const TG* beta, float* state, TQ* o, int n_seqs, int n_tokens,
                                  int n_heads, cudaStream_t stream) {
-  const unsigned chains = (unsigned)n_seqs * (unsigned)n_heads;
-  const size_t smem = sizeof(DecTokensSmem);
-  const cudaError_t e = cudaFuncSetAttribute(kda_decode_tokens_kernel<TQ, TG>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int chains = n_seqs * n_heads;
+  const size_t smem = dec_tokens_smem_bytes(n_tokens);
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kda_decode_tokens_kernel<TQ, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
   if (e != cudaSuccess) return e;
-  kda_decode_tokens_kernel<TQ, TG><<<chains, DEC_THREADS, smem, stream>>>(
-      q, k, v, log_alpha, beta, state, o, n_heads, n_tokens);
+  const int grid = chains < 2 * sms ? chains : 2 * sms;
+  kda_decode_tokens_kernel<TQ, TG><<<grid, DEC_THREADS, smem, stream>>>(
+      q, k, v, log_alpha, beta, state, o, n_heads, n_tokens, chains);
   return cudaGetLastError();
 }
 

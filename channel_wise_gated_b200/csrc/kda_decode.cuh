@@ -142,13 +142,26 @@ __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint3
 // Dynamic shared memory of the multi-token step, in bytes, for n_tokens tokens: the state
 // buffer, its barrier, the tokens' k, q, alpha, v in fp32, the partial projections and the
 // reduced delta double-buffered by token parity, beta and k.q.
-__host__ __device__ constexpr size_t dec_tokens_smem_bytes(int n_tokens) {
+// With input prefetch, the next chain's inputs arrive raw (q, k, v in their storage type,
+// log alpha in the gates' type) into a buffer of their own by 16-byte asynchronous copies.
+__host__ __device__ constexpr size_t dec_tokens_raw_bytes(int n_tokens, size_t q_bytes, size_t g_bytes) {
+  return (size_t)n_tokens * D * (3 * q_bytes + g_bytes);
+}
+__host__ __device__ constexpr size_t dec_tokens_smem_bytes(int n_tokens, size_t q_bytes, size_t g_bytes,
+                                                           bool prefetch) {
   return DEC_STATE_BYTES + 16 + (size_t)4 * n_tokens * D * sizeof(float) +
          2 * 2 * (DEC_THREADS / 32) * 32 * sizeof(float4) + 2 * D * sizeof(float) +
-         2 * DEC_MAX_TOKENS * sizeof(float);
+         2 * DEC_MAX_TOKENS * sizeof(float) +
+         (prefetch ? dec_tokens_raw_bytes(n_tokens, q_bytes, g_bytes) : 0);
 }
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_u32(dst_smem)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-template <typename TQ, typename TG>
+template <typename TQ, typename TG, bool PF>
 __global__ void __launch_bounds__(DEC_THREADS, 2)
 kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
                          const TQ* __restrict__ v, const TG* __restrict__ log_alpha,
@@ -170,7 +183,38 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
   float (*s_dl)[D] = reinterpret_cast<float (*)[D]>(s_y + 2);
   float* s_beta = reinterpret_cast<float*>(s_dl + 2);
   float* s_kq = s_beta + DEC_MAX_TOKENS;
+  unsigned char* raw = reinterpret_cast<unsigned char*>(s_kq + DEC_MAX_TOKENS);   // 16-byte aligned
+  TQ* r_q = reinterpret_cast<TQ*>(raw);
+  TQ* r_k = r_q + n_tokens * D;
+  TQ* r_v = r_k + n_tokens * D;
+  TG* r_a = reinterpret_cast<TG*>(r_v + n_tokens * D);
   const int row0 = warp * DEC_ROWS_PER_WARP;
+  // the inputs of chain ch: every (tensor, token) row of D elements is contiguous; 16-byte
+  // pieces, all threads, one commit group. beta (n_tokens scalars) goes to a register.
+  constexpr int QP = D * sizeof(TQ) / 16, GP = D * sizeof(TG) / 16;   // pieces per row
+  auto prefetch_inputs = [&](int ch, float& beta_r) {
+    const int sq = ch / n_heads, hd = ch - sq * n_heads;
+    const int nq = n_tokens * QP, ng = n_tokens * GP;
+#pragma unroll 1
+    for (int i = tid; i < 3 * nq + ng; i += DEC_THREADS) {
+      const int tensor = i < 3 * nq ? i / nq : 3;
+      const int j = tensor < 3 ? i - tensor * nq : i - 3 * nq;
+      const int per = tensor < 3 ? QP : GP;
+      const int t = j / per, piece = j - t * per;
+      const size_t row = ((size_t)sq * n_tokens + t) * n_heads + hd;
+      if (tensor < 3) {
+        const TQ* src = (tensor == 0 ? q : tensor == 1 ? k : v) + row * D;
+        TQ* dst = (tensor == 0 ? r_q : tensor == 1 ? r_k : r_v) + t * D;
+        cp_async16(reinterpret_cast<unsigned char*>(dst) + 16 * piece,
+                   reinterpret_cast<const unsigned char*>(src) + 16 * piece);
+      } else {
+        cp_async16(reinterpret_cast<unsigned char*>(r_a + t * D) + 16 * piece,
+                   reinterpret_cast<const unsigned char*>(log_alpha + row * D) + 16 * piece);
+      }
+    }
+    cp_async_commit();
+    beta_r = tid < n_tokens ? to_f32(beta[((size_t)sq * n_tokens + tid) * n_heads + hd]) : 0.f;
+  };
 
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -182,20 +226,42 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
     mbar_arrive_expect_tx(bar, DEC_STATE_BYTES);
     bulk_load(dec_smem, state + (size_t)chain * D * D, DEC_STATE_BYTES, bar);
   }
+  float beta_next = 0.f;
+  if constexpr (PF) {
+    if (chain < n_chains) prefetch_inputs(chain, beta_next);
+  }
   uint32_t phase = 0;
 #pragma unroll 1
   for (; chain < n_chains; chain += gridDim.x) {
     const int seq = chain / n_heads, h = chain - seq * n_heads;
+    if constexpr (PF) {
+      // this chain's inputs, copied while the previous chain computed: to fp32 (alpha
+      // from its log), then the buffer takes the next chain's
+      cp_async_wait_all();
+      __syncthreads();
 #pragma unroll 1
-    for (int i = tid; i < n_tokens * D; i += DEC_THREADS) {
-      const int t = i / D, c = i - t * D;
-      const size_t base = (((size_t)seq * n_tokens + t) * n_heads + h) * D + c;
-      s_k[i] = to_f32(k[base]);
-      s_q[i] = to_f32(q[base]);
-      s_v[i] = to_f32(v[base]);
-      s_a[i] = expf(to_f32(log_alpha[base]));
+      for (int i = tid; i < n_tokens * D; i += DEC_THREADS) {
+        s_k[i] = to_f32(r_k[i]);
+        s_q[i] = to_f32(r_q[i]);
+        s_v[i] = to_f32(r_v[i]);
+        s_a[i] = expf(to_f32(r_a[i]));
+      }
+      if (tid < n_tokens) s_beta[tid] = beta_next;
+      __syncthreads();
+      if (chain + (int)gridDim.x < n_chains) prefetch_inputs(chain + gridDim.x, beta_next);
+    } else {
+      // this chain's inputs, loaded now (read after the barrier below)
+#pragma unroll 1
+      for (int i = tid; i < n_tokens * D; i += DEC_THREADS) {
+        const int t = i / D, c = i - t * D;
+        const size_t base = (((size_t)seq * n_tokens + t) * n_heads + h) * D + c;
+        s_k[i] = to_f32(k[base]);
+        s_q[i] = to_f32(q[base]);
+        s_v[i] = to_f32(v[base]);
+        s_a[i] = expf(to_f32(log_alpha[base]));
+      }
+      if (tid < n_tokens) s_beta[tid] = to_f32(beta[((size_t)seq * n_tokens + tid) * n_heads + h]);
     }
-    if (tid < n_tokens) s_beta[tid] = to_f32(beta[((size_t)seq * n_tokens + tid) * n_heads + h]);
     // this chain's state, copied into the buffer while the previous chain computed
     const bool landed = mbar_wait(bar, phase);
     phase ^= 1u;
@@ -237,9 +303,9 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
       const float* sk_t = s_k + t * D;
       const float* sq_t = s_q + t * D;
       // decay and the two partial projections over this warp's rows (4 rows of the
-      // gates and keys per 16-byte read; rows in the single step's order)
-      float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+      // gates and keys per 16-byte read; rows in the single step's order). Two columns
+      // per instruction: the paired multiply and FMA round each lane as the scalar ones do.
+      float2 u0 = make_float2(0.f, 0.f), u1 = u0, y0 = u0, y1 = u0;
 #pragma unroll
       for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
         const float4 a4 = *reinterpret_cast<const float4*>(&sa_t[row0 + i4]);
@@ -250,16 +316,17 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = i4 + e;
-          const float a = av[e], kr = kv[e], qr = qv[e];
-          s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
-          u.x = fmaf(kr, s[i].x, u.x); u.y = fmaf(kr, s[i].y, u.y);
-          u.z = fmaf(kr, s[i].z, u.z); u.w = fmaf(kr, s[i].w, u.w);
-          y.x = fmaf(qr, s[i].x, y.x); y.y = fmaf(qr, s[i].y, y.y);
-          y.z = fmaf(qr, s[i].z, y.z); y.w = fmaf(qr, s[i].w, y.w);
+          const float2 a2 = make_float2(av[e], av[e]), k2 = make_float2(kv[e], kv[e]),
+                       q2 = make_float2(qv[e], qv[e]);
+          const float2 lo = __fmul2_rn(make_float2(s[i].x, s[i].y), a2);
+          const float2 hi = __fmul2_rn(make_float2(s[i].z, s[i].w), a2);
+          s[i] = make_float4(lo.x, lo.y, hi.x, hi.y);
+          u0 = __ffma2_rn(k2, lo, u0); u1 = __ffma2_rn(k2, hi, u1);
+          y0 = __ffma2_rn(q2, lo, y0); y1 = __ffma2_rn(q2, hi, y1);
         }
       }
-      s_u[buf][warp][lane] = u;
-      s_y[buf][warp][lane] = y;
+      s_u[buf][warp][lane] = make_float4(u0.x, u0.y, u1.x, u1.y);
+      s_y[buf][warp][lane] = make_float4(y0.x, y0.y, y1.x, y1.y);
       // (this token's buffers were last read two tokens ago, before the previous barriers)
       __syncthreads();
 
@@ -280,6 +347,7 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
       }
       __syncthreads();
       const float4 dl = reinterpret_cast<const float4*>(s_dl[buf])[lane];
+      const float2 dl0 = make_float2(dl.x, dl.y), dl1 = make_float2(dl.z, dl.w);
 #pragma unroll
       for (int i4 = 0; i4 < DEC_ROWS_PER_WARP; i4 += 4) {
         const float4 k4 = *reinterpret_cast<const float4*>(&sk_t[row0 + i4]);
@@ -287,9 +355,10 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = i4 + e;
-          const float kr = kv[e];
-          s[i].x = fmaf(kr, dl.x, s[i].x); s[i].y = fmaf(kr, dl.y, s[i].y);
-          s[i].z = fmaf(kr, dl.z, s[i].z); s[i].w = fmaf(kr, dl.w, s[i].w);
+          const float2 k2 = make_float2(kv[e], kv[e]);
+          const float2 lo = __ffma2_rn(k2, dl0, make_float2(s[i].x, s[i].y));
+          const float2 hi = __ffma2_rn(k2, dl1, make_float2(s[i].z, s[i].w));
+          s[i] = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
       }
     }
@@ -300,24 +369,43 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
 }
 
 // Host side: two persistent CTAs per SM (or one per state, if fewer); returns the
-// launch's CUDA error.
+// launch's CUDA error. The next chain's inputs are prefetched from three tokens on, as
+// long as two CTAs with the larger shared-memory layout still fit an SM: with one or two
+// tokens a chain is bound by its state copies, and the prefetch's extra barriers cost
+// more than the latency it hides.
+template <typename TQ, typename TG, bool PF>
+cudaError_t launch_decode_tokens_as(const TQ* q, const TQ* k, const TQ* v, const TG* log_alpha,
+                                    const TG* beta, float* state, TQ* o, int n_tokens,
+                                    int n_heads, int chains, int sms, cudaStream_t stream) {
+  const size_t smem = dec_tokens_smem_bytes(n_tokens, sizeof(TQ), sizeof(TG), PF);
+  cudaError_t e = cudaFuncSetAttribute(kda_decode_tokens_kernel<TQ, TG, PF>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = chains < 2 * sms ? chains : 2 * sms;
+  kda_decode_tokens_kernel<TQ, TG, PF><<<grid, DEC_THREADS, smem, stream>>>(
+      q, k, v, log_alpha, beta, state, o, n_heads, n_tokens, chains);
+  return cudaGetLastError();
+}
+
 template <typename TQ, typename TG>
 cudaError_t launch_decode_tokens(const TQ* q, const TQ* k, const TQ* v, const TG* log_alpha,
                                  const TG* beta, float* state, TQ* o, int n_seqs, int n_tokens,
                                  int n_heads, cudaStream_t stream) {
   const int chains = n_seqs * n_heads;
-  const size_t smem = dec_tokens_smem_bytes(n_tokens);
-  int dev = 0, sms = 0;
+  int dev = 0, sms = 0, smem_sm = 0, reserved = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kda_decode_tokens_kernel<TQ, TG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
   if (e != cudaSuccess) return e;
-  const int grid = chains < 2 * sms ? chains : 2 * sms;
-  kda_decode_tokens_kernel<TQ, TG><<<grid, DEC_THREADS, smem, stream>>>(
-      q, k, v, log_alpha, beta, state, o, n_heads, n_tokens, chains);
-  return cudaGetLastError();
+  const size_t pf_smem = dec_tokens_smem_bytes(n_tokens, sizeof(TQ), sizeof(TG), true);
+  if (n_tokens >= 3 && 2 * (pf_smem + (size_t)reserved) <= (size_t)smem_sm)
+    return launch_decode_tokens_as<TQ, TG, true>(q, k, v, log_alpha, beta, state, o, n_tokens,
+                                                 n_heads, chains, sms, stream);
+  return launch_decode_tokens_as<TQ, TG, false>(q, k, v, log_alpha, beta, state, o, n_tokens,
+                                                n_heads, chains, sms, stream);
 }
 
 }  // namespace kda

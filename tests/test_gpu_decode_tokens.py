@@ -87,6 +87,28 @@ def test_decode_tokens_equals_single_steps(kda, t, gates):
     assert torch.equal(s_multi, s_step)
 
 
+@pytest.mark.parametrize("t,qkv,gates", [(2, torch.bfloat16, torch.bfloat16),
+                                          (4, torch.bfloat16, torch.float32),
+                                          (4, torch.float32, torch.float32),
+                                          (9, torch.float32, torch.bfloat16),
+                                          (12, torch.bfloat16, torch.bfloat16)])
+def test_decode_tokens_many_chains_equal_single_steps(kda, t, qkv, gates):
+    """More (sequence, head) states than resident CTAs, so every CTA runs several in turn:
+    with and without the next state's input prefetch (the launcher prefetches from three
+    tokens on while two CTAs still fit an SM: not at t = 2, nor at t = 9 with fp32
+    inputs, nor at t = 12), still bit-identical to single steps."""
+    dec, lay = _draw(40, 16, t, qkv, gates, seed=160 + t)
+    s_multi = dec["state"].clone()
+    o_multi = kda.decode_tokens(lay["q"], lay["k"], lay["v"], lay["log_alpha"], lay["beta"],
+                                s_multi)
+    s_step = dec["state"].clone()
+    o_step = torch.stack([kda.decode_step(dec["q"][s], dec["k"][s], dec["v"][s],
+                                          dec["log_alpha"][s], dec["beta"][s], s_step)
+                          for s in range(t)], dim=1)
+    assert torch.equal(o_multi, o_step)
+    assert torch.equal(s_multi, s_step)
+
+
 def test_decode_tokens_full_batch(kda):
     """The multi-token decode workload that bench.py times: 256 sequences x 32 heads,
     4 tokens per call, 3 calls in a row; oracle on 48 sampled chains."""

@@ -4,12 +4,16 @@
 // projection, short convolution, Swish"). For token t of a sequence starting at bos,
 //     y_t[c] = swish( sum_{i=0..3} w[c][i] x_{t-3+i}[c] ),   x_s = 0 for s < bos,
 // swish(u) = u * sigmoid(u). Streaming and HBM-bound: every input row is read once
-// (plus a 3-row halo per run of tokens) and every output row written once.
+// (plus a 3-row halo per run of tokens, mostly from L2) and every output row written
+// once. At ~20 instructions per element the issue rate is close to the bandwidth too,
+// so the swish takes the fast division.
 //
 // Layout: x, y [T, C] bf16 (C a multiple of 8, e.g. H * 128), w [C, 4] fp32.
 // Thread = 8 channels (one 16-byte vector) x a run of CONV_RUN consecutive tokens; a
 // warp covers 256 consecutive channels of the same token, so its loads and stores of a
-// row are contiguous 512-byte segments. The three previous rows stay in registers.
+// row are contiguous 512-byte segments. The three previous rows stay in registers, and
+// the rows are loaded CONV_BATCH at a time ahead of their use, so that every thread has
+// that many 16-byte loads in flight (one at a time leaves HBM mostly idle).
 #pragma once
 
 #include "kda_common.cuh"
@@ -18,7 +22,8 @@ namespace kda {
 namespace conv {
 
 constexpr int CONV_THREADS = 256;
-constexpr int CONV_RUN = 32;   // tokens per thread
+constexpr int CONV_RUN = 32;     // tokens per thread
+constexpr int CONV_BATCH = 8;    // rows in flight per thread
 constexpr int TAPS = 4;
 
 __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
@@ -74,47 +79,56 @@ kda_short_conv_swish_kernel(const __nv_bfloat16* __restrict__ x, const float* __
     if (next > t_total) next = t_total;
     if (bos < 0) bos = 0;
   }
-  // the three rows before the run (zero before the sequence's first token)
+  // The stream of rows starts up to three rows before the run (not before the
+  // sequence's first token), which only fill the history; zero history before that.
+  const int64_t t_first = t_begin - 3 > bos ? t_begin - 3 : (bos < t_begin ? bos : t_begin);
   float h[3][8];
 #pragma unroll
-  for (int k = 0; k < 3; ++k) {
-    const int64_t s = t_begin - 3 + k;
-    if (s >= bos && s >= 0) {
-      unpack8(*reinterpret_cast<const uint4*>(x + (size_t)s * channels + c0), h[k]);
-    } else {
+  for (int k = 0; k < 3; ++k)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) h[k][i] = 0.f;
-    }
-  }
-  for (int64_t t = t_begin; t < t_end; ++t) {
-    while (t >= next && cu_seqlens != nullptr) {   // a new sequence: no history
-      ++n;
-      next = n + 1 <= n_seqs ? (int64_t)cu_seqlens[n + 1] : t_total;
-      if (next > t_total || next < t) next = next < t ? t + 1 : t_total;
+    for (int i = 0; i < 8; ++i) h[k][i] = 0.f;
+#pragma unroll 1
+  for (int64_t tb = t_first; tb < t_end; tb += CONV_BATCH) {
+    uint4 raw[CONV_BATCH];
 #pragma unroll
-      for (int k = 0; k < 3; ++k)
+    for (int b = 0; b < CONV_BATCH; ++b)
+      raw[b] = tb + b < t_end ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)(tb + b) * channels + c0))
+                              : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) h[k][i] = 0.f;
-    }
-    float cur[8];
-    unpack8(*reinterpret_cast<const uint4*>(x + (size_t)t * channels + c0), cur);
-    float out[8];
+    for (int b = 0; b < CONV_BATCH; ++b) {
+      const int64_t t = tb + b;
+      if (t >= t_end) break;
+      while (t >= next && cu_seqlens != nullptr) {   // a new sequence: no history
+        ++n;
+        next = n + 1 <= n_seqs ? (int64_t)cu_seqlens[n + 1] : t_total;
+        if (next > t_total || next < t) next = next < t ? t + 1 : t_total;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float u = wt[i][3] * cur[i];
-      u = fmaf(wt[i][2], h[2][i], u);
-      u = fmaf(wt[i][1], h[1][i], u);
-      u = fmaf(wt[i][0], h[0][i], u);
-      out[i] = u / (1.f + __expf(-u));   // swish
-    }
-    *reinterpret_cast<uint4*>(y + (size_t)t * channels + c0) =
-        make_uint4(pack2(out[0], out[1]), pack2(out[2], out[3]), pack2(out[4], out[5]),
-                   pack2(out[6], out[7]));
+        for (int k = 0; k < 3; ++k)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      h[0][i] = h[1][i];
-      h[1][i] = h[2][i];
-      h[2][i] = cur[i];
+          for (int i = 0; i < 8; ++i) h[k][i] = 0.f;
+      }
+      float cur[8];
+      unpack8(raw[b], cur);
+      if (t >= t_begin) {
+        float out[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float u = wt[i][3] * cur[i];
+          u = fmaf(wt[i][2], h[2][i], u);
+          u = fmaf(wt[i][1], h[1][i], u);
+          u = fmaf(wt[i][0], h[0][i], u);
+          out[i] = __fdividef(u, 1.f + __expf(-u));   // swish (0 where exp(-u) overflows)
+        }
+        __stcs(reinterpret_cast<uint4*>(y + (size_t)t * channels + c0),
+               make_uint4(pack2(out[0], out[1]), pack2(out[2], out[3]), pack2(out[4], out[5]),
+                          pack2(out[6], out[7])));
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        h[0][i] = h[1][i];
+        h[1][i] = h[2][i];
+        h[2][i] = cur[i];
+      }
     }
   }
 }

@@ -270,6 +270,7 @@ kda_decode_tokens_kernel(const TQ* __restrict__ q, const TQ* __restrict__ k,
     for (int i = 0; i < DEC_ROWS_PER_WARP; ++i) s[i] = sbuf[(row0 + i) * (D / 4) + lane];
     fence_proxy_async_smem();   // (these reads come before the next copy into the buffer)
     if (!__syncthreads_and(landed)) {   // (also the barrier before the staged inputs are read)
+      if constexpr (PF) cp_async_wait_all();   // (nor with the next inputs' copies in flight)
       if (tid == 0) {
         flag_error(DEVERR_TIMEOUT);
         mbar_wait(bar, phase ^ 1u, 100000000ull);   // (never leave with the copy in flight)

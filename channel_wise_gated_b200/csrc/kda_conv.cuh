@@ -23,7 +23,7 @@ namespace conv {
 
 constexpr int CONV_THREADS = 256;
 constexpr int CONV_RUN = 32;     // tokens per thread
-constexpr int CONV_BATCH = 8;    // rows in flight per thread
+constexpr int CONV_BATCH = 12;   // rows in flight per thread
 constexpr int TAPS = 4;
 
 __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {

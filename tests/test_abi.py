@@ -127,6 +127,52 @@ def test_chunk_validation(lib):
               None, None) == _native.KDA_ERR_ALIGN
 
 
+def test_layer_entry_points_validation(lib):
+    """The Gated DeltaNet, fused, general-DPLR and short-convolution entry points reject bad
+    arguments on the host, before any CUDA call."""
+    bf, f32 = _native.KDA_BF16, _native.KDA_F32
+    gdn, gdn_ws = lib.kda_gdn_chunk_fwd, lib.kda_gdn_chunk_fwd_ws
+    assert gdn(None, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, bf, FAKE, None,
+               None) == _native.KDA_ERR_NULL
+    assert gdn(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, 5, FAKE, None,
+               None) == _native.KDA_ERR_DTYPE
+    assert gdn(FAKE, FAKE, FAKE, FAKE + 4, FAKE, None, None, 1, 64, 2, bf, FAKE, None,
+               None) == _native.KDA_ERR_ALIGN
+    assert gdn_ws(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 2, bf, FAKE, None, FAKE + 8,
+                  1 << 20, None) == _native.KDA_ERR_ALIGN
+    assert gdn_ws(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 3, 64, 2, bf, FAKE, None, None, 0,
+                  None) == _native.KDA_ERR_SEQLENS
+    # fused: q_pre, k_pre, v, decay_pre, beta_pre, gate_pre, norm_w, h0, cu, n, T, H, o, hT, ws
+    fused = lambda **a: lib.kda_chunk_fwd_fused(
+        a.get("q", FAKE), FAKE, FAKE, FAKE, FAKE, a.get("gate", FAKE), a.get("norm", FAKE), None,
+        None, 1, 64, a.get("H", 2), FAKE, None, a.get("ws", None), 0, None)
+    assert fused(q=None) == _native.KDA_ERR_NULL
+    assert fused(gate=None) == _native.KDA_ERR_NULL
+    assert fused(norm=None) == _native.KDA_ERR_NULL
+    assert fused(gate=FAKE + 2) == _native.KDA_ERR_ALIGN
+    assert fused(ws=FAKE + 8) == _native.KDA_ERR_ALIGN
+    assert fused(H=0) == _native.KDA_ERR_SHAPE
+    # general DPLR: q, k, v, a, b, log_alpha, h0, cu, n, T, H, dtype, o, hT
+    dplr = lambda **x: lib.kda_dplr_chunk_fwd(
+        FAKE, FAKE, FAKE, x.get("a", FAKE), x.get("b", FAKE), FAKE, None, None, 1, 64, 2,
+        x.get("dt", f32), FAKE, None, None)
+    assert dplr(a=None) == _native.KDA_ERR_NULL
+    assert dplr(b=FAKE + 4) == _native.KDA_ERR_ALIGN
+    assert dplr(dt=9) == _native.KDA_ERR_DTYPE
+    # short convolution: x, w, cu, n_seqs, T, channels, y
+    conv = lambda **x: lib.kda_short_conv_swish(
+        x.get("x", FAKE), x.get("w", FAKE), x.get("cu", None), x.get("n", 1), x.get("T", 64),
+        x.get("C", 256), x.get("y", FAKE + 4096), None)
+    assert conv(C=12) == _native.KDA_ERR_SHAPE        # not a multiple of 8 channels
+    assert conv(C=0) == _native.KDA_ERR_SHAPE
+    assert conv(T=-1) == _native.KDA_ERR_SHAPE
+    assert conv(n=2) == _native.KDA_ERR_SEQLENS       # several sequences need cu_seqlens
+    assert conv(x=None) == _native.KDA_ERR_NULL
+    assert conv(w=FAKE + 4) == _native.KDA_ERR_ALIGN
+    assert conv(y=FAKE) == _native.KDA_ERR_SHAPE      # no in-place convolution
+    assert conv(T=0, x=None, w=None, y=None) == _native.KDA_OK   # nothing to do
+
+
 def test_workspace_size_queries(lib):
     size = lib.kda_chunk_fwd_workspace_size
     bf, f32 = _native.KDA_BF16, _native.KDA_F32
